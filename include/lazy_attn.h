@@ -1,0 +1,212 @@
+/*
+ * lazy_attn.h -- C ABI of a B200 (sm_100a) library for LazyAttention's hot
+ * path: attention over a shared, paged KV cache whose keys are stored with
+ * RoPE at document-local positions, with each request's document offsets
+ * applied inside the kernels.
+ *
+ * Sources (three web pages about arXiv 2606.04302):
+ *   [ABS] shd-paper.top, "LazyAttention: Efficient Retrieval-Augmented
+ *         Generation with Deferred Positional Encoding" -- English abstract.
+ *   [CORE], [PRE], [DEC], [EQV], [CON]: gist.science, same title --
+ *         Technical Summary: Core Concept: Deferred Positional Encoding;
+ *         Technical Implementation: Prefilling; Technical Implementation:
+ *         Decoding; Mathematical Equivalence; Key Contributions.
+ *
+ * Conventions for every entry point
+ *   - Pointers are DEVICE pointers unless marked "host".  bf16 tensors are
+ *     passed as uint16_t bit patterns.  `stream` is a cudaStream_t (NULL =
+ *     the legacy default stream).  Every launch is asynchronous on it.
+ *   - Ownership: the caller allocates and frees every buffer (pools, tables,
+ *     outputs, workspaces).  The library allocates no device memory and keeps
+ *     no state between calls.
+ *   - Errors found on the host (bad shapes, null pointers, a workspace too
+ *     small) are returned BEFORE anything is launched.  A launch failure
+ *     returns LAZY_ECUDA.
+ *   - Errors found on the device (a block id >= num_blocks, a slot outside
+ *     the pool, a segment that is not block-aligned, a bounded wait that ran
+ *     out) are OR-ed into *d_status (a device int, may be NULL) as
+ *     LAZY_DSTATUS_* bits; the affected unit of work is skipped (its output
+ *     rows are written as zeros, or its pool slot is not written).  Nothing
+ *     traps.
+ *
+ * Data layout
+ *   - Pools: k_pool, v_pool are bf16 [num_blocks][Hkv][16][head_dim]; one
+ *     16-token block of one KV head is 4 KiB contiguous.  Keys are stored as
+ *     RoPE(k, j) at their local index j inside their segment ([CORE]; the
+ *     pages leave open what is stored and the plainest reading consistent
+ *     with a "single relative rotation" [PRE] is the local position).
+ *   - blk_meta: uint32 [num_blocks], one word per physical block:
+ *     (j0 / 16) << 8 | n_valid, with j0 the local index of the block's first
+ *     token and n_valid (1..16) the number of written slots.  lazy_kv_write
+ *     maintains it; the caller zeroes the words of freshly allocated blocks.
+ *   - Tables: per request r, table[table_indptr[r] .. table_indptr[r+1]) holds
+ *     one 32-bit word per logical block, in logical order:
+ *         word = (offset << 17) | block
+ *     block = physical block id (17 bits), offset = logical offset of the
+ *     block's segment in tokens (15 bits) ([DEC]: "(block ID, offset)
+ *     bit-packed into a single register").  Slot s of the block holds local
+ *     index j0 + s and sits at logical position offset + j0 + s.  The same
+ *     physical block may appear in many requests and several times in one
+ *     request at different offsets; gaps between segments are legal.
+ *   - Queries: bf16 [tokens][Hq][head_dim], unrotated.  Outputs: bf16, same
+ *     shape.  Query head h reads KV head h / (Hq / Hkv) ([CON]: GQA/MQA).
+ *   - Causal rule: a key at logical position t is visible to a query at
+ *     position p iff t <= p.  A query that sees no key gets a zero row.
+ *   - head_dim must be 128 and block_size 16.  Hq / Hkv must be an integer
+ *     <= 32.
+ */
+#ifndef LAZY_ATTN_H
+#define LAZY_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct lazy_attn_cfg {
+    int num_q_heads;     /* Hq */
+    int num_kv_heads;    /* Hkv; Hq % Hkv == 0, Hq / Hkv <= 32 */
+    int head_dim;        /* must be 128 */
+    int block_size;      /* must be 16 */
+    float rope_base;     /* RoPE base, e.g. 500000; theta_i = base^(-2i/d) */
+    float softmax_scale; /* <= 0 selects 1/sqrt(head_dim) */
+} lazy_attn_cfg;
+
+/* Host-side return codes. */
+enum {
+    LAZY_OK = 0,
+    LAZY_EINVAL = -1,     /* null pointer or negative count */
+    LAZY_ERANGE = -2,     /* a table field overflows 17/15 bits, or a size is too large */
+    LAZY_ESHAPE = -3,     /* head_dim != 128, block_size != 16, bad head counts */
+    LAZY_EWORKSPACE = -4, /* workspace smaller than the matching *_workspace_bytes() */
+    LAZY_ECUDA = -5       /* a CUDA launch or driver call failed */
+};
+
+/* Device-side status bits, OR-ed into *d_status. */
+enum {
+    LAZY_DSTATUS_BAD_BLOCK = 1,   /* a table word names a block >= num_blocks */
+    LAZY_DSTATUS_BAD_SLOT = 2,    /* lazy_kv_write: slot outside the pool */
+    LAZY_DSTATUS_BAD_ALIGN = 4,   /* lazy_kv_write: local index j and slot differ mod 16 */
+    LAZY_DSTATUS_BAD_TABLE = 8,   /* a request has more words than max_words */
+    LAZY_DSTATUS_TIMEOUT = 16     /* a bounded pipeline wait ran out (kernel bailed out) */
+};
+
+#define LAZY_BLOCK_BITS 17
+#define LAZY_OFFSET_BITS 15
+#define LAZY_MAX_BLOCKS (1u << LAZY_BLOCK_BITS)
+#define LAZY_MAX_OFFSET ((1u << LAZY_OFFSET_BITS) - 1u)
+
+/* Table-word codec, usable from host and device code.  No range check:
+ * callers that cannot guarantee block < 2^17 and offset < 2^15 use
+ * lazy_pack_words, which checks. */
+static inline uint32_t lazy_pack(uint32_t block, uint32_t offset) { return (offset << LAZY_BLOCK_BITS) | block; }
+static inline uint32_t lazy_block(uint32_t word) { return word & (LAZY_MAX_BLOCKS - 1u); }
+static inline uint32_t lazy_offset(uint32_t word) { return word >> LAZY_BLOCK_BITS; }
+
+/* Packs n (block, offset) pairs into table words.  HOST pointers.
+ * Returns LAZY_ERANGE (and stops) at the first field that does not fit. */
+int lazy_pack_words(const int32_t *block, const int32_t *offset, int64_t n, uint32_t *words);
+
+/* Writes n_tok tokens' keys and values into the paged pools ([CORE], [ABS]):
+ *   k_pool[slot/16][h][slot%16][:] = bf16_rne(RoPE(k_raw[t][h][:], local_j[t]))
+ *   v_pool[slot/16][h][slot%16][:] = v_raw[t][h][:]
+ *   blk_meta[slot/16] = max(blk_meta[slot/16], (local_j/16) << 8 | (slot%16 + 1))
+ * k_raw, v_raw: bf16 [n_tok][Hkv][128], unrotated.  slot, local_j: int32 [n_tok].
+ * RoPE is computed in fp32 with angles reduced in fp64.  A slot outside the
+ * pool (LAZY_DSTATUS_BAD_SLOT) or with local_j % 16 != slot % 16
+ * (LAZY_DSTATUS_BAD_ALIGN) is skipped.  Distinct tokens must use distinct slots. */
+int lazy_kv_write(const lazy_attn_cfg *cfg, const uint16_t *k_raw, const uint16_t *v_raw, int n_tok,
+                  const int32_t *slot, const int32_t *local_j, uint16_t *k_pool, uint16_t *v_pool,
+                  uint32_t *blk_meta, int num_blocks, int *d_status, void *stream);
+
+/* Workspace for lazy_decode_attn: split-K partial results. */
+size_t lazy_decode_workspace_bytes(const lazy_attn_cfg *cfg, int num_req, int max_words);
+
+/* One decode step: one query token per request over its table ([DEC]).
+ * q_raw: bf16 [num_req][Hq][128]; q_pos: int32 [num_req] (the query's logical
+ * position; its own key must already be in the pool, written by
+ * lazy_kv_write).  max_words: host upper bound of words per request (sizes the
+ * split-K grid and the workspace; a request with more words sets
+ * LAZY_DSTATUS_BAD_TABLE).  out: bf16 [num_req][Hq][128].
+ * The query is rotated by (q_pos - offset) in registers whenever a warp
+ * meets a new segment offset; keys are used as stored, so the kernel reads
+ * only K and V ([DEC]: "memory traffic remains identical to the baseline").
+ * Two launches: split-K attention, then a combine over splits. */
+int lazy_decode_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *q_pos, int num_req,
+                     const uint32_t *table, const int32_t *table_indptr, int max_words,
+                     const uint32_t *blk_meta, const uint16_t *k_pool, const uint16_t *v_pool,
+                     int num_blocks, uint16_t *out, void *workspace, size_t ws_bytes, int *d_status,
+                     void *stream);
+
+/* Workspace for lazy_prefill_attn. */
+size_t lazy_prefill_workspace_bytes(const lazy_attn_cfg *cfg, int num_req, int total_q, int max_q,
+                                    int max_words);
+
+/* Causal prefill of a chunk of query tokens per request over its table ([PRE]).
+ * q_raw: bf16 [total_q][Hq][128]; request r owns tokens cu_q[r] .. cu_q[r+1]-1
+ * at positions q_pos0[r] + i.  max_q: host upper bound of tokens per request;
+ * max_words as for decode.  out: bf16 [total_q][Hq][128].
+ * For each segment the query tile is rotated once by (p_i - offset): one
+ * relative rotation, not a reset to position 0 and a re-rotation. */
+int lazy_prefill_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *cu_q,
+                      const int32_t *q_pos0, int num_req, int total_q, int max_q,
+                      const uint32_t *table, const int32_t *table_indptr, int max_words,
+                      const uint32_t *blk_meta, const uint16_t *k_pool, const uint16_t *v_pool,
+                      int num_blocks, uint16_t *out, void *workspace, size_t ws_bytes, int *d_status,
+                      void *stream);
+
+/* ---- comparison paths (the position-aware alternative the pages argue against) ---- */
+
+/* Materialises position-adjusted keys ([ABS]: "memory materialization for
+ * positional re-encoding"): for every table word w (global index into table,
+ * 0 <= w < total_words) with block b and offset o,
+ *   k_mat[w][h][s][:] = bf16_rne(RoPE(k_pool[b][h][s][:], o))   for s < n_valid(b)
+ *   k_mat[w][h][s][:] = 0                                        otherwise
+ * i.e. keys rotated to their absolute positions o + j.  k_mat: bf16
+ * [total_words][Hkv][16][128]. */
+int lazy_materialize_k(const lazy_attn_cfg *cfg, const uint32_t *table, int total_words,
+                       const uint32_t *blk_meta, const uint16_t *k_pool, int num_blocks,
+                       uint16_t *k_mat, int *d_status, void *stream);
+
+/* Plain paged attention over materialised keys: the same kernels with the
+ * deferred rotation removed.  Keys come from k_mat (indexed by the word's
+ * global table index, as written by lazy_materialize_k), values from v_pool
+ * (indexed by the word's block), and the query is rotated once, at its
+ * absolute position.  Arguments otherwise as lazy_decode_attn /
+ * lazy_prefill_attn, whose workspace sizes apply. */
+int lazy_plain_decode_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *q_pos,
+                           int num_req, const uint32_t *table, const int32_t *table_indptr,
+                           int max_words, const uint32_t *blk_meta, const uint16_t *k_mat,
+                           int total_words, const uint16_t *v_pool, int num_blocks, uint16_t *out,
+                           void *workspace, size_t ws_bytes, int *d_status, void *stream);
+
+int lazy_plain_prefill_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *cu_q,
+                            const int32_t *q_pos0, int num_req, int total_q, int max_q,
+                            const uint32_t *table, const int32_t *table_indptr, int max_words,
+                            const uint32_t *blk_meta, const uint16_t *k_mat, int total_words,
+                            const uint16_t *v_pool, int num_blocks, uint16_t *out, void *workspace,
+                            size_t ws_bytes, int *d_status, void *stream);
+
+/* ---- test export ---- */
+
+/* Decodes n_words table words on the device, exactly as the attention kernels
+ * do, into per-slot records: out_block[16w+s] = block, out_slot[16w+s] =
+ * 16*block + s, out_pos[16w+s] = offset + j0 + s if s < n_valid else -1.
+ * A block id >= num_blocks gives -1 records and LAZY_DSTATUS_BAD_BLOCK. */
+int lazy_debug_decode_table(const uint32_t *table, int64_t n_words, const uint32_t *blk_meta,
+                            int num_blocks, int32_t *out_block, int32_t *out_slot, int32_t *out_pos,
+                            int *d_status, void *stream);
+
+/* Text for a host return code (static storage). */
+const char *lazy_strerror(int code);
+
+/* Library ABI version (major * 100 + minor). */
+int lazy_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LAZY_ATTN_H */

@@ -1,0 +1,80 @@
+// kernels.h -- parameter blocks and launch entry points shared between the
+// host ABI layer (abi.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lazy_attn.h"
+
+namespace lazy {
+
+struct RopeTableHost {
+    double theta[64];
+};
+
+struct KvWriteParams {
+    const uint16_t *k_raw, *v_raw;
+    const int32_t *slot, *local_j;
+    uint16_t *k_pool, *v_pool;
+    uint32_t *blk_meta;
+    int n_tok, hkv, num_blocks;
+    int *d_status;
+    RopeTableHost rope;
+};
+
+struct DecodeTableParams {
+    const uint32_t *table;
+    int64_t n_words;
+    const uint32_t *blk_meta;
+    int num_blocks;
+    int32_t *out_block, *out_slot, *out_pos;
+    int *d_status;
+};
+
+struct MaterializeParams {
+    const uint32_t *table;
+    const uint32_t *blk_meta;
+    const uint16_t *k_pool;
+    uint16_t *k_mat;
+    int total_words, hkv, num_blocks;
+    int *d_status;
+    RopeTableHost rope;
+};
+
+struct AttnParams {
+    const uint16_t *q_raw;
+    const int32_t *q_pos;        // decode: [B] query position
+    const int32_t *cu_q;         // prefill: [B+1]
+    const int32_t *q_pos0;       // prefill: [B]
+    const uint32_t *table;
+    const int32_t *table_indptr;
+    const uint32_t *blk_meta;
+    uint16_t *out;
+    float *ws_acc;               // decode: [B][Hkv][S][G][128]
+    float *ws_ml;                // decode: [B][Hkv][S][G][2]
+    int *d_status;
+    int num_req, hq, hkv, group, num_blocks, max_words;
+    int words_per_split, n_splits;   // decode
+    int max_q;                       // prefill
+    float scale_log2;            // softmax scale * log2(e)
+    RopeTableHost rope;
+};
+
+// Decode split plan shared by the workspace query and the launch.
+struct DecodePlan {
+    int words_per_split;
+    int n_splits;
+};
+DecodePlan decode_plan(int num_req, int hkv, int max_words);
+
+cudaError_t launch_kv_write(const KvWriteParams &p, cudaStream_t s);
+cudaError_t launch_decode_table(const DecodeTableParams &p, cudaStream_t s);
+cudaError_t launch_materialize(const MaterializeParams &p, cudaStream_t s);
+cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, bool plain,
+                          cudaStream_t s);
+cudaError_t launch_prefill(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, bool plain,
+                           cudaStream_t s);
+
+}  // namespace lazy

@@ -1,0 +1,199 @@
+"""Thin ctypes binding of liblazy_attn.so (include/lazy_attn.h).
+
+Argument marshalling only: every function takes torch tensors that already
+live on the GPU, passes their data pointers and the current CUDA stream to the
+C entry point of the same name, and raises LazyAttnError on a non-zero return
+code.  All computation happens in the library's CUDA kernels; there is no CPU
+fallback, and importing this module fails loudly when the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblazy_attn.so")
+
+LAZY_OK, LAZY_EINVAL, LAZY_ERANGE, LAZY_ESHAPE, LAZY_EWORKSPACE, LAZY_ECUDA = 0, -1, -2, -3, -4, -5
+DSTATUS_BAD_BLOCK, DSTATUS_BAD_SLOT, DSTATUS_BAD_ALIGN, DSTATUS_BAD_TABLE, DSTATUS_TIMEOUT = 1, 2, 4, 8, 16
+
+EXPORTED = [
+    "lazy_version", "lazy_strerror", "lazy_pack_words", "lazy_kv_write",
+    "lazy_decode_workspace_bytes", "lazy_decode_attn",
+    "lazy_prefill_workspace_bytes", "lazy_prefill_attn",
+    "lazy_materialize_k", "lazy_plain_decode_attn", "lazy_plain_prefill_attn",
+    "lazy_debug_decode_table",
+]
+
+
+class LazyAttnError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {code}: {strerror(code)}")
+        self.code = code
+
+
+class LazyAttnCfg(ctypes.Structure):
+    _fields_ = [("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("block_size", ctypes.c_int), ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float)]
+
+
+@dataclass(frozen=True)
+class Cfg:
+    num_q_heads: int
+    num_kv_heads: int
+    rope_base: float = 500000.0
+    head_dim: int = 128
+    block_size: int = 16
+    softmax_scale: float = 0.0
+
+    def c(self) -> LazyAttnCfg:
+        return LazyAttnCfg(self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
+                           float(self.rope_base), float(self.softmax_scale))
+
+
+_vp, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+_cfgp = ctypes.POINTER(LazyAttnCfg)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m position_agnostic_paged_b200.build` "
+                          "(the CUDA library is required; there is no fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "lazy_version": (_i, []),
+        "lazy_strerror": (ctypes.c_char_p, [_i]),
+        "lazy_pack_words": (_i, [_vp, _vp, _i64, _vp]),
+        "lazy_kv_write": (_i, [_cfgp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp]),
+        "lazy_decode_workspace_bytes": (_sz, [_cfgp, _i, _i]),
+        "lazy_decode_attn": (_i, [_cfgp, _vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _sz, _vp, _vp]),
+        "lazy_prefill_workspace_bytes": (_sz, [_cfgp, _i, _i, _i, _i]),
+        "lazy_prefill_attn": (_i, [_cfgp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp,
+                                   _sz, _vp, _vp]),
+        "lazy_materialize_k": (_i, [_cfgp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp]),
+        "lazy_plain_decode_attn": (_i, [_cfgp, _vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _i, _vp, _i, _vp, _vp, _sz,
+                                        _vp, _vp]),
+        "lazy_plain_prefill_attn": (_i, [_cfgp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _vp, _vp, _i, _vp, _i,
+                                         _vp, _vp, _sz, _vp, _vp]),
+        "lazy_debug_decode_table": (_i, [_vp, _i64, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def version() -> int:
+    return int(_lib.lazy_version())
+
+
+def strerror(code: int) -> str:
+    return _lib.lazy_strerror(int(code)).decode()
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != 0:
+        raise LazyAttnError(fn, rc)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    return int(t.data_ptr())
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream) or None
+    return int(getattr(stream, "cuda_stream", stream)) or None
+
+
+def pack_words(block: np.ndarray, offset: np.ndarray) -> np.ndarray:
+    """Host codec: (block, offset) int32 arrays -> uint32 table words (raises on overflow)."""
+    block = np.ascontiguousarray(block, np.int32)
+    offset = np.ascontiguousarray(offset, np.int32)
+    out = np.empty(block.size, np.uint32)
+    _check("lazy_pack_words", _lib.lazy_pack_words(block.ctypes.data, offset.ctypes.data, block.size,
+                                                   out.ctypes.data))
+    return out
+
+
+def kv_write(cfg: Cfg, k_raw, v_raw, slot, local_j, k_pool, v_pool, blk_meta, d_status=None, stream=None):
+    c = cfg.c()
+    _check("lazy_kv_write", _lib.lazy_kv_write(
+        ctypes.byref(c), _ptr(k_raw), _ptr(v_raw), int(slot.numel()), _ptr(slot), _ptr(local_j),
+        _ptr(k_pool), _ptr(v_pool), _ptr(blk_meta), int(k_pool.shape[0]), _ptr(d_status), _stream(stream)))
+
+
+def decode_workspace_bytes(cfg: Cfg, num_req: int, max_words: int) -> int:
+    c = cfg.c()
+    return int(_lib.lazy_decode_workspace_bytes(ctypes.byref(c), int(num_req), int(max_words)))
+
+
+def prefill_workspace_bytes(cfg: Cfg, num_req: int, total_q: int, max_q: int, max_words: int) -> int:
+    c = cfg.c()
+    return int(_lib.lazy_prefill_workspace_bytes(ctypes.byref(c), int(num_req), int(total_q), int(max_q),
+                                                 int(max_words)))
+
+
+def decode_attn(cfg: Cfg, q_raw, q_pos, table, table_indptr, max_words: int, blk_meta, k_pool, v_pool, out,
+                workspace, d_status=None, stream=None):
+    c = cfg.c()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("lazy_decode_attn", _lib.lazy_decode_attn(
+        ctypes.byref(c), _ptr(q_raw), _ptr(q_pos), int(q_pos.numel()), _ptr(table), _ptr(table_indptr),
+        int(max_words), _ptr(blk_meta), _ptr(k_pool), _ptr(v_pool), int(k_pool.shape[0]), _ptr(out),
+        _ptr(workspace), ws_bytes, _ptr(d_status), _stream(stream)))
+
+
+def prefill_attn(cfg: Cfg, q_raw, cu_q, q_pos0, max_q: int, table, table_indptr, max_words: int, blk_meta,
+                 k_pool, v_pool, out, workspace=None, d_status=None, stream=None):
+    c = cfg.c()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("lazy_prefill_attn", _lib.lazy_prefill_attn(
+        ctypes.byref(c), _ptr(q_raw), _ptr(cu_q), _ptr(q_pos0), int(q_pos0.numel()), int(q_raw.shape[0]),
+        int(max_q), _ptr(table), _ptr(table_indptr), int(max_words), _ptr(blk_meta), _ptr(k_pool),
+        _ptr(v_pool), int(k_pool.shape[0]), _ptr(out), _ptr(workspace), ws_bytes, _ptr(d_status),
+        _stream(stream)))
+
+
+def materialize_k(cfg: Cfg, table, blk_meta, k_pool, k_mat, d_status=None, stream=None):
+    c = cfg.c()
+    _check("lazy_materialize_k", _lib.lazy_materialize_k(
+        ctypes.byref(c), _ptr(table), int(table.numel()), _ptr(blk_meta), _ptr(k_pool), int(k_pool.shape[0]),
+        _ptr(k_mat), _ptr(d_status), _stream(stream)))
+
+
+def plain_decode_attn(cfg: Cfg, q_raw, q_pos, table, table_indptr, max_words: int, blk_meta, k_mat, v_pool, out,
+                      workspace, d_status=None, stream=None):
+    c = cfg.c()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("lazy_plain_decode_attn", _lib.lazy_plain_decode_attn(
+        ctypes.byref(c), _ptr(q_raw), _ptr(q_pos), int(q_pos.numel()), _ptr(table), _ptr(table_indptr),
+        int(max_words), _ptr(blk_meta), _ptr(k_mat), int(k_mat.shape[0]), _ptr(v_pool), int(v_pool.shape[0]),
+        _ptr(out), _ptr(workspace), ws_bytes, _ptr(d_status), _stream(stream)))
+
+
+def plain_prefill_attn(cfg: Cfg, q_raw, cu_q, q_pos0, max_q: int, table, table_indptr, max_words: int, blk_meta,
+                       k_mat, v_pool, out, workspace=None, d_status=None, stream=None):
+    c = cfg.c()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("lazy_plain_prefill_attn", _lib.lazy_plain_prefill_attn(
+        ctypes.byref(c), _ptr(q_raw), _ptr(cu_q), _ptr(q_pos0), int(q_pos0.numel()), int(q_raw.shape[0]),
+        int(max_q), _ptr(table), _ptr(table_indptr), int(max_words), _ptr(blk_meta), _ptr(k_mat),
+        int(k_mat.shape[0]), _ptr(v_pool), int(v_pool.shape[0]), _ptr(out), _ptr(workspace), ws_bytes,
+        _ptr(d_status), _stream(stream)))
+
+
+def debug_decode_table(table, blk_meta, num_blocks: int, out_block, out_slot, out_pos, d_status=None, stream=None):
+    _check("lazy_debug_decode_table", _lib.lazy_debug_decode_table(
+        _ptr(table), int(table.numel()), _ptr(blk_meta), int(num_blocks), _ptr(out_block), _ptr(out_slot),
+        _ptr(out_pos), _ptr(d_status), _stream(stream)))

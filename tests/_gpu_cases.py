@@ -1,0 +1,112 @@
+"""Device set-up of hand-shaped cases (tests/_cases.Case) for GPU parity tests.
+
+Each distinct source range of the case's token store becomes one document
+stored once in the paged pool (its tokens at local indices 0..len-1); every
+segment that uses it becomes table words (block, offset).  Two segments with
+the same source therefore share one physical copy, as in the pages' zero-copy
+reuse.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from position_agnostic_paged_b200 import lazy_attn as la
+
+
+def _u16(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+
+def _i32(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a, np.int32)).to(dev)
+
+
+class DeviceCase:
+    def __init__(self, case, dev="cuda", extra_blocks: int = 0):
+        self.case = case
+        self.cfg = la.Cfg(case.hq, case.hkv, rope_base=case.base)
+        docs = {}
+        for g in range(case.seg_src.size):
+            src, ln = int(case.seg_src[g]), int(case.seg_len[g])
+            assert docs.get(src, ln) == ln, "a source must always be used with the same length"
+            docs[src] = ln
+        self.doc_block = {}
+        nb = 0
+        for src in sorted(docs):
+            self.doc_block[src] = nb
+            nb += (docs[src] + 15) // 16
+        self.num_blocks = nb + extra_blocks
+        shape = (max(self.num_blocks, 1), case.hkv, 16, case.d)
+        self.k_pool = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+        self.v_pool = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+        self.blk_meta = torch.zeros(shape[0], dtype=torch.int32, device=dev)
+        self.d_status = torch.zeros(1, dtype=torch.int32, device=dev)
+        rows, slots, js = [], [], []
+        for src, ln in docs.items():
+            for j in range(ln):
+                rows.append(src + j)
+                slots.append(self.doc_block[src] * 16 + j)
+                js.append(j)
+        if rows:
+            la.kv_write(self.cfg, _u16(case.k_tok[rows], dev), _u16(case.v_tok[rows], dev), _i32(slots, dev),
+                        _i32(js, dev), self.k_pool, self.v_pool, self.blk_meta, self.d_status)
+        blocks, offs, indptr = [], [], [0]
+        for r in range(case.cu_q.size - 1):
+            for g in range(case.seg_indptr[r], case.seg_indptr[r + 1]):
+                src, off, ln = int(case.seg_src[g]), int(case.seg_off[g]), int(case.seg_len[g])
+                for k in range((ln + 15) // 16):
+                    blocks.append(self.doc_block[src] + k)
+                    offs.append(off)
+            indptr.append(len(blocks))
+        self.words = la.pack_words(np.array(blocks, np.int32), np.array(offs, np.int32))
+        self.table = torch.from_numpy(self.words.view(np.int32).copy()).to(dev)
+        self.table_indptr = _i32(indptr, dev)
+        self.max_words = int(np.diff(indptr).max()) if len(indptr) > 1 else 0
+        self.dev = dev
+
+    def decode(self, plain: bool = False):
+        c = self.case
+        n = c.cu_q.size - 1
+        assert np.array_equal(np.diff(c.cu_q), np.ones(n)), "decode: one query per request"
+        out = torch.zeros((n, c.hq, c.d), dtype=torch.bfloat16, device=self.dev)
+        ws = torch.empty(max(16, la.decode_workspace_bytes(self.cfg, n, self.max_words)), dtype=torch.uint8,
+                         device=self.dev)
+        q = _u16(c.q_raw, self.dev)
+        qp = _i32(c.q_pos, self.dev)
+        if plain:
+            kmat = torch.empty((self.table.numel(), c.hkv, 16, c.d), dtype=torch.bfloat16, device=self.dev)
+            la.materialize_k(self.cfg, self.table, self.blk_meta, self.k_pool, kmat, self.d_status)
+            la.plain_decode_attn(self.cfg, q, qp, self.table, self.table_indptr, self.max_words, self.blk_meta,
+                                 kmat, self.v_pool, out, ws, self.d_status)
+        else:
+            la.decode_attn(self.cfg, q, qp, self.table, self.table_indptr, self.max_words, self.blk_meta,
+                           self.k_pool, self.v_pool, out, ws, self.d_status)
+        return out.float().cpu().numpy().astype(np.float64).reshape(-1, c.d)
+
+    def prefill(self, plain: bool = False):
+        c = self.case
+        n = c.cu_q.size - 1
+        q_pos0 = []
+        for r in range(n):
+            qp = c.q_pos[c.cu_q[r]:c.cu_q[r + 1]]
+            assert np.array_equal(qp, qp[0] + np.arange(qp.size)), "prefill: contiguous query positions"
+            q_pos0.append(int(qp[0]) if qp.size else 0)
+        total_q = int(c.cu_q[-1])
+        max_q = int(np.diff(c.cu_q).max())
+        out = torch.zeros((total_q, c.hq, c.d), dtype=torch.bfloat16, device=self.dev)
+        q = _u16(c.q_raw, self.dev)
+        cu = _i32(c.cu_q, self.dev)
+        p0 = _i32(q_pos0, self.dev)
+        if plain:
+            kmat = torch.empty((self.table.numel(), c.hkv, 16, c.d), dtype=torch.bfloat16, device=self.dev)
+            la.materialize_k(self.cfg, self.table, self.blk_meta, self.k_pool, kmat, self.d_status)
+            la.plain_prefill_attn(self.cfg, q, cu, p0, max_q, self.table, self.table_indptr, self.max_words,
+                                  self.blk_meta, kmat, self.v_pool, out, None, self.d_status)
+        else:
+            la.prefill_attn(self.cfg, q, cu, p0, max_q, self.table, self.table_indptr, self.max_words,
+                            self.blk_meta, self.k_pool, self.v_pool, out, None, self.d_status)
+        return out.float().cpu().numpy().astype(np.float64).reshape(-1, c.d)
+
+    def status(self) -> int:
+        return int(self.d_status.item())

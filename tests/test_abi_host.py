@@ -1,0 +1,89 @@
+"""The C-ABI library loads, exports every symbol its header declares, and its
+host-side logic (word codec, argument validation, workspace sizing) behaves as
+documented.  Nothing here launches a kernel, so it runs without a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from position_agnostic_paged_b200 import lazy_attn as la
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "lazy_attn.h")
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?(?:int|size_t|char\s*\*|void)\s*\*?\s*(lazy_\w+)\s*\(", txt, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert len(names) >= 12
+    lib = ctypes.CDLL(la.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in lazy_attn.h but not exported"
+    assert sorted(la.EXPORTED) == names
+
+
+def test_version_and_strerror():
+    assert la.version() == 100
+    for code in (0, -1, -2, -3, -4, -5):
+        assert la.strerror(code) and la.strerror(code) != "unknown error"
+
+
+def test_pack_words_bit_exact_against_oracle():
+    rng = np.random.default_rng(0)
+    b = np.concatenate([[0, 131071, 0, 131071], rng.integers(0, 131072, 1000)]).astype(np.int32)
+    o = np.concatenate([[0, 0, 32767, 32767], rng.integers(0, 32768, 1000)]).astype(np.int32)
+    got = la.pack_words(b, o)
+    ref = np.array([oracle.pack_word(int(x), int(y)) for x, y in zip(b, o)], np.uint32)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("b,o", [(131072, 0), (0, 32768), (-1, 0), (0, -5)])
+def test_pack_words_rejects_overflow(b, o):
+    with pytest.raises(la.LazyAttnError) as e:
+        la.pack_words(np.array([1, b], np.int32), np.array([1, o], np.int32))
+    assert e.value.code == la.LAZY_ERANGE
+
+
+def _call_decode(cfg, **kw):
+    c = cfg.c()
+    args = dict(q=1, qp=1, n=2, table=1, indptr=1, maxw=4, meta=1, k=1, v=1, nb=8, out=1, ws=1, wsb=1 << 20)
+    args.update(kw)
+    return la._lib.lazy_decode_attn(ctypes.byref(c), args["q"], args["qp"], args["n"], args["table"],
+                                    args["indptr"], args["maxw"], args["meta"], args["k"], args["v"], args["nb"],
+                                    args["out"], args["ws"], args["wsb"], None, None)
+
+
+def test_host_validation_returns_before_launch():
+    ok = la.Cfg(8, 2)
+    assert _call_decode(la.Cfg(8, 2, head_dim=64)) == la.LAZY_ESHAPE
+    assert _call_decode(la.Cfg(8, 3)) == la.LAZY_ESHAPE
+    assert _call_decode(la.Cfg(64, 1)) == la.LAZY_ESHAPE          # G = 64 > 32
+    assert _call_decode(la.Cfg(8, 2, block_size=32)) == la.LAZY_ESHAPE
+    assert _call_decode(ok, q=None) == la.LAZY_EINVAL
+    assert _call_decode(ok, n=-1) == la.LAZY_EINVAL
+    assert _call_decode(ok, nb=(1 << 17) + 1) == la.LAZY_ERANGE
+    assert _call_decode(ok, wsb=16) == la.LAZY_EWORKSPACE
+    assert _call_decode(ok, ws=None) == la.LAZY_EWORKSPACE
+    c = ok.c()
+    assert la._lib.lazy_kv_write(None, 1, 1, 1, 1, 1, 1, 1, 1, 8, None, None) == la.LAZY_EINVAL
+    assert la._lib.lazy_kv_write(ctypes.byref(c), None, 1, 1, 1, 1, 1, 1, 1, 8, None, None) == la.LAZY_EINVAL
+    assert la._lib.lazy_materialize_k(ctypes.byref(c), None, 4, 1, 1, 8, 1, None, None) == la.LAZY_EINVAL
+    assert la._lib.lazy_debug_decode_table(None, 4, 1, 8, 1, 1, 1, None, None) == la.LAZY_EINVAL
+
+
+def test_decode_workspace_sizes():
+    cfg = la.Cfg(32, 8)
+    a = la.decode_workspace_bytes(cfg, 64, 261)
+    b = la.decode_workspace_bytes(cfg, 1, 261)
+    assert 0 < b < a
+    # one (m, l, acc[128]) record of fp32 per (request, kv head, split, head in group)
+    assert a % ((128 + 2) * 4 * 4) == 0
+    assert la.decode_workspace_bytes(la.Cfg(32, 8, head_dim=64), 64, 261) == 0

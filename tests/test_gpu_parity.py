@@ -1,0 +1,239 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Tolerances (floating point): max |gpu - ref| <= 1e-2 and
+||gpu - ref||_2 / ||ref||_2 <= 5e-3 over the compared outputs.  Integer work
+(table decoding, pool indexing, block metadata) is bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from position_agnostic_paged_b200 import lazy_attn as la
+from position_agnostic_paged_b200 import workloads as W
+from position_agnostic_paged_b200.runner import DevicePool, DeviceStep
+from tests._cases import bits_to_f64, make_case
+from tests._gpu_cases import DeviceCase
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 1e-2
+REL_L2 = 5e-3
+
+
+def check(got, ref, max_abs=MAX_ABS, rel_l2=REL_L2, what=""):
+    assert np.isfinite(got).all(), f"{what}: non-finite GPU output"
+    err = np.abs(got - ref)
+    ma = float(err.max()) if err.size else 0.0
+    rl = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+    assert ma <= max_abs and rl <= rel_l2, f"{what}: max_abs={ma:.3e} rel_l2={rl:.3e}"
+    return ma, rl
+
+
+def oracle_step(wl, step, sel_q=None, sel_h=None):
+    return oracle.attend(num_q_heads=wl.hq, num_kv_heads=wl.hkv, rope_base=wl.rope_base, q_raw=step.q_raw,
+                         cu_q=step.cu_q, q_pos=step.q_pos, seg_indptr=step.seg_indptr, seg_src=step.seg_src,
+                         seg_off=step.seg_off, seg_len=step.seg_len, k_tok=wl.k_store, v_tok=wl.v_store,
+                         sel_q=sel_q, sel_h=sel_h)
+
+
+# ----------------------------------------------------------------------------- tiny workload
+def test_tiny_prefill_then_decode_lazy_and_plain():
+    wl = W.make("tiny")
+    pool = DevicePool(wl).setup()
+    for step in wl.steps:
+        ds = DeviceStep(pool, step, with_plain=True)
+        ds.write_new_tokens()
+        ds.attend()
+        ds.materialize()
+        ds.attend_plain()
+        torch.cuda.synchronize()
+        ref = oracle_step(wl, step)
+        lazy = ds.out_f64()
+        plain = ds.out_f64(ds.out_plain)
+        check(lazy, ref, what=f"{step.kind} lazy")
+        check(plain, ref, what=f"{step.kind} plain")
+        check(lazy, plain, what=f"{step.kind} lazy vs plain")
+    assert pool.status() == 0
+
+
+def test_pool_contents_and_metadata_bit_exact():
+    wl = W.make("tiny")
+    pool = DevicePool(wl, sentinel=-1).setup()
+    for step in wl.steps:
+        pool.write_rows(step.write_rows)
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    kp = np.full((wl.num_blocks, wl.hkv, 16, wl.d), 0xFFFF, np.uint16)
+    vp = kp.copy()
+    meta = np.zeros(wl.num_blocks, np.uint32)
+    rows = np.concatenate([wl.setup_rows] + [s.write_rows for s in wl.steps])
+    assert oracle.kv_write(wl.k_store[rows], wl.v_store[rows], wl.store_slot[rows], wl.store_j[rows],
+                           kp, vp, meta, wl.rope_base) == 0
+    gk = pool.k_pool.view(torch.int16).cpu().numpy().view(np.uint16)
+    gv = pool.v_pool.view(torch.int16).cpu().numpy().view(np.uint16)
+    gm = pool.blk_meta.cpu().numpy().view(np.uint32)
+    assert np.array_equal(gm, meta), "block metadata"
+    assert np.array_equal(gv, vp), "values: placement and copy"
+    written = np.zeros((wl.num_blocks, 16), bool)
+    written.reshape(-1)[wl.store_slot[rows]] = True
+    # untouched slots keep the sentinel in both pools
+    assert (gk[~written] == 0xFFFF).all() and (gv[~written] == 0xFFFF).all()
+    # j = 0 slots are identity rotations: exact copies of the raw keys
+    j0 = rows[wl.store_j[rows] == 0]
+    s0 = wl.store_slot[j0]
+    assert np.array_equal(gk[s0 // 16, :, s0 % 16], wl.k_store[j0])
+    # every rotated key within one bf16 ulp of the correctly rounded fp64 rotation
+    diff = np.abs(gk.astype(np.int32) - kp.astype(np.int32))
+    assert diff[written].max() <= 1, f"max ulp difference {diff[written].max()}"
+    assert (diff[written] != 0).mean() < 0.02
+
+
+def test_table_decoding_bit_exact():
+    wl = W.make("tiny")
+    pool = DevicePool(wl).setup()
+    for step in wl.steps:
+        pool.write_rows(step.write_rows)
+    step = wl.steps[-1]
+    ds = DeviceStep(pool, step)
+    n = ds.table.numel()
+    ob = torch.empty(n * 16, dtype=torch.int32, device="cuda")
+    osl, op = torch.empty_like(ob), torch.empty_like(ob)
+    la.debug_decode_table(ds.table, pool.blk_meta, wl.num_blocks, ob, osl, op, pool.d_status)
+    # oracle side: its own word packing and its own expected metadata
+    words = np.array([oracle.pack_word(b, o) for b, o in zip(step.table_block, step.table_off)], np.uint32)
+    assert np.array_equal(words, ds.words_np)
+    meta = np.zeros(wl.num_blocks, np.uint32)
+    kp = np.zeros((wl.num_blocks, wl.hkv, 16, wl.d), np.uint16)
+    rows = np.concatenate([wl.setup_rows] + [s.write_rows for s in wl.steps])
+    oracle.kv_write(wl.k_store[rows], wl.v_store[rows], wl.store_slot[rows], wl.store_j[rows], kp, kp.copy(),
+                    meta, wl.rope_base)
+    eb, es, epos, rc = oracle.expand_table(words, meta, wl.num_blocks)
+    assert rc == 0
+    assert np.array_equal(ob.cpu().numpy(), eb.ravel())
+    assert np.array_equal(osl.cpu().numpy(), es.ravel())
+    assert np.array_equal(op.cpu().numpy(), epos.ravel())
+    # the logical positions seen through the table are exactly the request's key positions
+    vis = epos[epos >= 0]
+    expect = np.concatenate([np.arange(o, o + L) for o, L in zip(step.seg_off, step.seg_len)])
+    assert np.array_equal(np.sort(vis), np.sort(expect))
+
+
+def test_bad_block_id_is_reported_and_isolated():
+    case = make_case(21, hq=8, hkv=2, d=128, requests=[([(0, 0, 40)], [39]), ([(40, 0, 24)], [23])])
+    dc = DeviceCase(case)
+    good = dc.decode()
+    words = dc.words.copy()
+    words[0] = la.pack_words(np.array([dc.num_blocks + 5], np.int32), np.array([0], np.int32))[0]
+    dc.table.copy_(torch.from_numpy(words.view(np.int32)))
+    out = dc.decode()
+    assert dc.status() & la.DSTATUS_BAD_BLOCK
+    np.testing.assert_array_equal(out[8:], good[8:])   # request 1 untouched
+
+
+# ----------------------------------------------------------------------------- adversarial small cases
+def _adv_requests(decode: bool):
+    # gaps, the same document (store rows 0..36) twice at two offsets, partial
+    # blocks (37, 7, 21, 5 tokens), a request whose query precedes some keys
+    segs0 = [(0, 0, 37), (40, 50, 7), (0, 60, 37), (50, 110, 21)]
+    segs1 = [(80, 3, 5), (0, 9, 37)]
+    if decode:
+        return [(segs0, [125]), (segs1, [20])]
+    return [(segs0, list(range(95, 131))), (segs1, list(range(0, 50)))]
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 2), (32, 8), (64, 8), (32, 1), (16, 1)])
+@pytest.mark.parametrize("kind", ["decode", "prefill"])
+def test_adversarial_cases_all_group_sizes(kind, hq, hkv):
+    case = make_case(100 + hq + hkv, hq=hq, hkv=hkv, d=128, requests=_adv_requests(kind == "decode"))
+    dc = DeviceCase(case)
+    ref = oracle.attend(**case.oracle_kwargs())
+    got = dc.decode() if kind == "decode" else dc.prefill()
+    check(got, ref, what=f"{kind} G={hq // hkv} lazy")
+    got_p = dc.decode(plain=True) if kind == "decode" else dc.prefill(plain=True)
+    check(got_p, ref, what=f"{kind} G={hq // hkv} plain")
+    assert dc.status() == 0
+
+
+def test_queries_that_see_nothing_give_zero_rows():
+    case = make_case(5, hq=8, hkv=2, d=128, requests=[([(0, 100, 20)], [50]), ([(20, 0, 16)], [15])])
+    dc = DeviceCase(case)
+    out = dc.decode()
+    assert np.array_equal(out[:8], np.zeros((8, 128)))
+    check(out[8:], oracle.attend(**case.oracle_kwargs())[8:])
+
+
+def test_peaked_scores():
+    # queries x4 (exact in bf16) make the softmax much sharper
+    case = make_case(9, hq=32, hkv=8, d=128, requests=_adv_requests(True))
+    qf = bits_to_f64(case.q_raw) * 4.0
+    case.q_raw = (qf.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    dc = DeviceCase(case)
+    ref = oracle.attend(**case.oracle_kwargs())
+    # score errors scale with |q|: bf16 rounding of q' and k (2^-9 relative
+    # each) on scores 4x larger; the bound below is 4x the base tolerance
+    check(dc.decode(), ref, max_abs=4e-2, rel_l2=2e-2, what="peaked decode")
+
+
+def test_decode_equals_last_prefill_row():
+    segs = [(0, 0, 64), (64, 64, 40)]
+    case = make_case(13, hq=32, hkv=8, d=128, requests=[(segs, list(range(64, 104)))])
+    dc = DeviceCase(case)
+    pf = dc.prefill()
+    last = make_case(13, hq=32, hkv=8, d=128, requests=[(segs, [103])])
+    last.k_tok, last.v_tok = case.k_tok, case.v_tok
+    last.q_raw = case.q_raw[-1:]
+    dl = DeviceCase(last).decode()
+    check(dl, pf[-32:], what="decode vs last prefill row")
+
+
+# ----------------------------------------------------------------------------- full-size configurations
+def _sample_rows(step, hq, n, seed):
+    rng = np.random.default_rng(seed)
+    q = rng.integers(0, step.total_q, n)
+    q[:2] = [0, step.total_q - 1]
+    h = rng.integers(0, hq, n)
+    h[:2] = [0, hq - 1]
+    return q.astype(np.int32), h.astype(np.int32)
+
+
+def _run_full(name, n_rows, **over):
+    wl = W.make(name, **over)
+    pool = DevicePool(wl).setup()
+    results = []
+    for step in wl.steps:
+        ds = DeviceStep(pool, step, with_plain=True)
+        ds.write_new_tokens()
+        ds.attend()
+        ds.materialize()
+        ds.attend_plain()
+        torch.cuda.synchronize()
+        sq, sh = _sample_rows(step, wl.hq, n_rows, 7)
+        ref = oracle_step(wl, step, sq, sh)
+        lazy = ds.out_f64().reshape(step.total_q, wl.hq, wl.d)
+        plain = ds.out_f64(ds.out_plain).reshape(step.total_q, wl.hq, wl.d)
+        check(lazy[sq, sh], ref, what=f"{name} {step.kind} sampled lazy")
+        check(plain[sq, sh], ref, what=f"{name} {step.kind} sampled plain")
+        # every row: lazy and materialised paths agree (a property that holds at any size)
+        check(lazy.reshape(-1, wl.d), plain.reshape(-1, wl.d), what=f"{name} {step.kind} lazy vs plain")
+        results.append(step.kind)
+    assert pool.status() == 0
+    return results
+
+
+def test_decode_8b_full_size():
+    assert _run_full("decode_8b", 64) == ["decode"]
+
+
+def test_prefill_8b_full_size():
+    assert _run_full("prefill_8b", 64) == ["prefill"]
+
+
+@pytest.mark.slow
+def test_decode_70b_full_size():
+    assert _run_full("decode_70b", 24) == ["decode"]
+
+
+@pytest.mark.slow
+def test_mixed_8b_mqa_full_size():
+    assert _run_full("mixed_8b_mqa", 32) == ["prefill", "decode"]
