@@ -304,7 +304,7 @@ def run_ours(args):
         plain_total, _ = timed_steps(plain_step, args.steps, args.warmup, flush, world)
         mat_total, _ = timed_steps(mat_step, args.steps, args.warmup, flush, world)
         torch.cuda.synchronize()
-        lazy_vs_plain = float(np.abs(ds.out.float() - ds.out_plain.float()).max().item())
+        lazy_vs_plain = float((ds.out.float() - ds.out_plain.float()).abs().max().item())
         result["comparison"] = {
             "lazy_decode_attn_ms": round(attn_avg, 5),
             "plain_decode_attn_ms": round(max_over_ranks(world, plain_total / args.steps), 5),

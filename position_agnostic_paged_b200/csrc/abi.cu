@@ -7,6 +7,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -126,6 +127,8 @@ int decode_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *
     const DecodePlan pl = decode_plan(num_req, cfg->num_kv_heads, max_words);
     p.q_raw = q_raw;
     p.q_pos = q_pos;
+    p.k_rows = static_cast<int>(k_rows);
+    p.v_rows = static_cast<int>(static_cast<int64_t>(num_blocks) * p.hkv * 16);
     p.words_per_split = pl.words_per_split;
     p.n_splits = pl.n_splits;
     const size_t parts = static_cast<size_t>(num_req) * p.hkv * pl.n_splits * p.group;
@@ -161,14 +164,15 @@ int prefill_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t 
     p.cu_q = cu_q;
     p.q_pos0 = q_pos0;
     p.max_q = max_q;
+    p.k_rows = static_cast<int>(k_rows);
+    p.v_rows = static_cast<int>(static_cast<int64_t>(num_blocks) * p.hkv * 16);
     CUtensorMap tk, tv;
-    if (!make_rows_map(&tk, k_src, k_rows) ||
-        !make_rows_map(&tv, v_pool, static_cast<int64_t>(num_blocks) * p.hkv * 16))
-        return LAZY_ECUDA;
-    // rows a request does not own are written by no CTA: zero them first so
-    // that a short request's tail is well defined is NOT needed -- each
-    // request writes exactly its own tokens.
-    return launch_rc(launch_prefill(tk, tv, p, plain, static_cast<cudaStream_t>(stream)));
+    if (!make_rows_map(&tk, k_src, k_rows) || !make_rows_map(&tv, v_pool, p.v_rows)) return LAZY_ECUDA;
+    // each request writes exactly its own query tokens' rows
+    const char *impl = getenv("LAZY_ATTN_PREFILL_IMPL");
+    if (impl && impl[0] == 'm')
+        return launch_rc(launch_prefill(tk, tv, p, plain, static_cast<cudaStream_t>(stream)));
+    return launch_rc(launch_prefill_tc(tk, tv, p, plain, static_cast<cudaStream_t>(stream)));
 }
 
 }  // namespace

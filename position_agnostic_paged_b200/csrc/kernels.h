@@ -58,6 +58,7 @@ struct AttnParams {
     int num_req, hq, hkv, group, num_blocks, max_words;
     int words_per_split, n_splits;   // decode
     int max_q;                       // prefill
+    int k_rows, v_rows;              // rows (of 128 bf16) covered by the K and V tensor maps
     float scale_log2;            // softmax scale * log2(e)
     RopeTableHost rope;
 };
@@ -76,5 +77,7 @@ cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const At
                           cudaStream_t s);
 cudaError_t launch_prefill(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, bool plain,
                            cudaStream_t s);
+cudaError_t launch_prefill_tc(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, bool plain,
+                              cudaStream_t s);
 
 }  // namespace lazy

@@ -21,6 +21,19 @@ MAX_ABS = 1e-2
 REL_L2 = 5e-3
 
 
+def edge_max_abs(case) -> float:
+    """Absolute bound for hand-made cases where a query may see only a few keys.
+
+    The kernels feed P to the PV product in bf16 (relative rounding <= 2^-9
+    per weight) and round the output to bf16 (<= 2^-9 |O|).  With few visible
+    keys O is close to single value rows, so the error is bounded by about
+    2^-9 (|O| + 2 max|V|) <= 3 * 2^-9 * max|V| -- the config-sized workloads,
+    where every query sees thousands of keys, keep the absolute 1e-2.
+    """
+    vmax = float(np.abs(bits_to_f64(case.v_tok)).max())
+    return max(MAX_ABS, 3 * 2.0 ** -9 * vmax)
+
+
 def check(got, ref, max_abs=MAX_ABS, rel_l2=REL_L2, what=""):
     assert np.isfinite(got).all(), f"{what}: non-finite GPU output"
     err = np.abs(got - ref)
@@ -77,16 +90,19 @@ def test_pool_contents_and_metadata_bit_exact():
     assert np.array_equal(gv, vp), "values: placement and copy"
     written = np.zeros((wl.num_blocks, 16), bool)
     written.reshape(-1)[wl.store_slot[rows]] = True
+    gk_s = gk.transpose(0, 2, 1, 3)    # [block, slot, head, d]
+    gv_s = gv.transpose(0, 2, 1, 3)
+    kp_s = kp.transpose(0, 2, 1, 3)
     # untouched slots keep the sentinel in both pools
-    assert (gk[~written] == 0xFFFF).all() and (gv[~written] == 0xFFFF).all()
+    assert (gk_s[~written] == 0xFFFF).all() and (gv_s[~written] == 0xFFFF).all()
     # j = 0 slots are identity rotations: exact copies of the raw keys
     j0 = rows[wl.store_j[rows] == 0]
     s0 = wl.store_slot[j0]
     assert np.array_equal(gk[s0 // 16, :, s0 % 16], wl.k_store[j0])
     # every rotated key within one bf16 ulp of the correctly rounded fp64 rotation
-    diff = np.abs(gk.astype(np.int32) - kp.astype(np.int32))
-    assert diff[written].max() <= 1, f"max ulp difference {diff[written].max()}"
-    assert (diff[written] != 0).mean() < 0.02
+    diff = np.abs(gk_s.astype(np.int32) - kp_s.astype(np.int32))[written]
+    assert diff.max() <= 1, f"max ulp difference {diff.max()}"
+    assert (diff != 0).mean() < 0.02
 
 
 def test_table_decoding_bit_exact():
@@ -148,10 +164,11 @@ def test_adversarial_cases_all_group_sizes(kind, hq, hkv):
     case = make_case(100 + hq + hkv, hq=hq, hkv=hkv, d=128, requests=_adv_requests(kind == "decode"))
     dc = DeviceCase(case)
     ref = oracle.attend(**case.oracle_kwargs())
+    tol = edge_max_abs(case)
     got = dc.decode() if kind == "decode" else dc.prefill()
-    check(got, ref, what=f"{kind} G={hq // hkv} lazy")
+    check(got, ref, max_abs=tol, what=f"{kind} G={hq // hkv} lazy")
     got_p = dc.decode(plain=True) if kind == "decode" else dc.prefill(plain=True)
-    check(got_p, ref, what=f"{kind} G={hq // hkv} plain")
+    check(got_p, ref, max_abs=tol, what=f"{kind} G={hq // hkv} plain")
     assert dc.status() == 0
 
 
@@ -160,7 +177,7 @@ def test_queries_that_see_nothing_give_zero_rows():
     dc = DeviceCase(case)
     out = dc.decode()
     assert np.array_equal(out[:8], np.zeros((8, 128)))
-    check(out[8:], oracle.attend(**case.oracle_kwargs())[8:])
+    check(out[8:], oracle.attend(**case.oracle_kwargs())[8:], max_abs=edge_max_abs(case))
 
 
 def test_peaked_scores():
@@ -172,7 +189,7 @@ def test_peaked_scores():
     ref = oracle.attend(**case.oracle_kwargs())
     # score errors scale with |q|: bf16 rounding of q' and k (2^-9 relative
     # each) on scores 4x larger; the bound below is 4x the base tolerance
-    check(dc.decode(), ref, max_abs=4e-2, rel_l2=2e-2, what="peaked decode")
+    check(dc.decode(), ref, max_abs=4 * edge_max_abs(case), rel_l2=2e-2, what="peaked decode")
 
 
 def test_decode_equals_last_prefill_row():
