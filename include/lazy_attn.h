@@ -18,7 +18,8 @@
  *     the legacy default stream).  Every launch is asynchronous on it.
  *   - Ownership: the caller allocates and frees every buffer (pools, tables,
  *     outputs, workspaces).  The library allocates no device memory and keeps
- *     no state between calls.
+ *     no state between calls, except the fixed scratch array that
+ *     lazy_decode_attn_noalloc uses (described at its declaration).
  *   - Errors found on the host (bad shapes, null pointers, a workspace too
  *     small) are returned BEFORE anything is launched.  A launch failure
  *     returns LAZY_ECUDA.
@@ -33,8 +34,8 @@
  *   - Pools: k_pool, v_pool are bf16 [num_blocks][Hkv][16][head_dim]; one
  *     16-token block of one KV head is 4 KiB contiguous.  Keys are stored as
  *     RoPE(k, j) at their local index j inside their segment ([CORE]; the
- *     pages leave open what is stored and the plainest reading consistent
- *     with a "single relative rotation" [PRE] is the local position).
+ *     pages leave open what is stored, and the local position is the plainest
+ *     reading that lets one relative rotation per segment suffice [PRE]).
  *   - blk_meta: uint32 [num_blocks], one word per physical block:
  *     (j0 / 16) << 8 | n_valid, with j0 the local index of the block's first
  *     token and n_valid (1..16) the number of written slots.  lazy_kv_write
@@ -43,8 +44,8 @@
  *     one 32-bit word per logical block, in logical order:
  *         word = (offset << 17) | block
  *     block = physical block id (17 bits), offset = logical offset of the
- *     block's segment in tokens (15 bits) ([DEC]: "(block ID, offset)
- *     bit-packed into a single register").  Slot s of the block holds local
+ *     block's segment in tokens (15 bits) ([DEC]: the block id and the offset
+ *     are packed together into one register word).  Slot s of the block holds local
  *     index j0 + s and sits at logical position offset + j0 + s.  The same
  *     physical block may appear in many requests and several times in one
  *     request at different offsets; gaps between segments are legal.
@@ -132,13 +133,37 @@ size_t lazy_decode_workspace_bytes(const lazy_attn_cfg *cfg, int num_req, int ma
  * LAZY_DSTATUS_BAD_TABLE).  out: bf16 [num_req][Hq][128].
  * The query is rotated by (q_pos - offset) in registers whenever a warp
  * meets a new segment offset; keys are used as stored, so the kernel reads
- * only K and V ([DEC]: "memory traffic remains identical to the baseline").
+ * only K and V ([DEC]: its memory traffic equals that of plain paged attention).
  * Two launches: split-K attention, then a combine over splits. */
 int lazy_decode_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *q_pos, int num_req,
                      const uint32_t *table, const int32_t *table_indptr, int max_words,
                      const uint32_t *blk_meta, const uint16_t *k_pool, const uint16_t *v_pool,
                      int num_blocks, uint16_t *out, void *workspace, size_t ws_bytes, int *d_status,
                      void *stream);
+
+/* lazy_decode_attn for callers that cannot allocate device memory.  The
+ * paper has no counterpart: this is a deployment convenience of this library.
+ * Some callers have no allocator to draw a workspace from (a plugin handed
+ * only its input and output buffers by a serving engine), or must not call
+ * cudaMalloc on their hot path because it synchronises the device.  This
+ * variant keeps the split-K partials in a fixed array inside the library's
+ * device image (lazy_decode_noalloc_capacity() bytes, 16 MiB, held by every
+ * GPU that loads the library until the process exits) and allocates nothing.
+ * Arguments and results are those of lazy_decode_attn minus the workspace.
+ * Returns LAZY_ERANGE, before launching anything, when the call needs more
+ * than the capacity (lazy_decode_workspace_bytes(cfg, num_req, max_words) >
+ * capacity).  The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress), so make that first call before any stream
+ * capture.  All calls share the array: calls that can overlap on the GPU
+ * (different streams or host threads) race and must be serialised by the
+ * caller. */
+int lazy_decode_attn_noalloc(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *q_pos, int num_req,
+                             const uint32_t *table, const int32_t *table_indptr, int max_words,
+                             const uint32_t *blk_meta, const uint16_t *k_pool, const uint16_t *v_pool,
+                             int num_blocks, uint16_t *out, int *d_status, void *stream);
+
+/* Bytes of the built-in scratch array used by lazy_decode_attn_noalloc. */
+size_t lazy_decode_noalloc_capacity(void);
 
 /* Workspace for lazy_prefill_attn. */
 size_t lazy_prefill_workspace_bytes(const lazy_attn_cfg *cfg, int num_req, int total_q, int max_q,

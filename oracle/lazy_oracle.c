@@ -36,8 +36,8 @@
  *     t <= p.  A query that sees no key produces a zero row.
  *   - GQA: query head h reads KV head h / G with G = Hq / Hkv ([CON]).
  *   - Table word: low 17 bits physical block id, high 15 bits the segment's
- *     logical offset in tokens ([DEC] says only "(block ID, offset)
- *     bit-packed into a single register").
+ *     logical offset in tokens ([DEC] states only that the block id and
+ *     the offset are packed together into one register word).
  *   - Block metadata word: (j0 / 16) << 8 | n_valid, where j0 is the local
  *     index of the block's first token inside its segment and n_valid (1..16)
  *     the number of written slots.
@@ -105,7 +105,7 @@ uint16_t oracle_f64_to_bf16(double x)
 }
 
 /* ------------------------------------------------------------------------- */
-/* Segment-table word codec ([DEC]: "(block ID, offset)" in one register).    */
+/* Segment-table word codec ([DEC]: block id and offset share one 32-bit word). */
 /* ------------------------------------------------------------------------- */
 
 int oracle_pack_word(int64_t block, int64_t offset, uint32_t *word)

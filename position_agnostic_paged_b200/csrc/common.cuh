@@ -150,8 +150,10 @@ __device__ __forceinline__ void set_status(int *d_status, int bits) {
     if (d_status) atomicOr(d_status, bits);
 }
 
-// Table word and block-metadata decoding, in registers ([DEC]: "(block ID,
-// offset) bit-packed into a single register").
+// Table word and block-metadata decoding, in registers.  The block id and the
+// segment offset share one 32-bit word (gist.science, "LazyAttention: Efficient
+// Retrieval-Augmented Generation with Deferred Positional Encoding", Technical
+// Summary, Technical Implementation: Decoding).
 __device__ __forceinline__ uint32_t word_block(uint32_t w) { return w & (LAZY_MAX_BLOCKS - 1u); }
 __device__ __forceinline__ int word_offset(uint32_t w) { return static_cast<int>(w >> LAZY_BLOCK_BITS); }
 __device__ __forceinline__ int meta_j0(uint32_t m) { return static_cast<int>(m >> 8) * kBlockTokens; }

@@ -6,7 +6,7 @@
 // Sources: gist.science, "LazyAttention: Efficient Retrieval-Augmented
 // Generation with Deferred Positional Encoding", Technical Summary: Core
 // Concept (deferred positional encoding) and Technical Implementation:
-// Decoding ("(block ID, offset)" bit-packed words); shd-paper.top, same
+// Decoding (block id and offset packed in one word); shd-paper.top, same
 // title, English abstract (materialisation of re-encoded copies is the cost
 // the method avoids).
 #include "common.cuh"

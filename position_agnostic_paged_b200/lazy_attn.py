@@ -25,7 +25,7 @@ EXPORTED = [
     "lazy_decode_workspace_bytes", "lazy_decode_attn",
     "lazy_prefill_workspace_bytes", "lazy_prefill_attn",
     "lazy_materialize_k", "lazy_plain_decode_attn", "lazy_plain_prefill_attn",
-    "lazy_debug_decode_table",
+    "lazy_debug_decode_table", "lazy_decode_attn_noalloc", "lazy_decode_noalloc_capacity",
 ]
 
 
@@ -79,6 +79,8 @@ def _load():
         "lazy_plain_prefill_attn": (_i, [_cfgp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _vp, _vp, _i, _vp, _i,
                                          _vp, _vp, _sz, _vp, _vp]),
         "lazy_debug_decode_table": (_i, [_vp, _i64, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
+        "lazy_decode_attn_noalloc": (_i, [_cfgp, _vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
+        "lazy_decode_noalloc_capacity": (_sz, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -197,3 +199,24 @@ def debug_decode_table(table, blk_meta, num_blocks: int, out_block, out_slot, ou
     _check("lazy_debug_decode_table", _lib.lazy_debug_decode_table(
         _ptr(table), int(table.numel()), _ptr(blk_meta), int(num_blocks), _ptr(out_block), _ptr(out_slot),
         _ptr(out_pos), _ptr(d_status), _stream(stream)))
+
+
+def decode_noalloc_capacity() -> int:
+    """Bytes of the library's built-in scratch array used by decode_attn_noalloc."""
+    return int(_lib.lazy_decode_noalloc_capacity())
+
+
+def decode_attn_noalloc(cfg: Cfg, q_raw, q_pos, table, table_indptr, max_words: int, blk_meta, k_pool, v_pool, out,
+                        d_status=None, stream=None):
+    """decode_attn without a workspace, for callers that cannot allocate device memory.
+
+    The split partials live in a fixed array inside the library (see
+    decode_noalloc_capacity()); calls that may overlap on the GPU must be
+    serialised by the caller.  Raises LazyAttnError(LAZY_ERANGE) when the
+    batch needs more scratch than the array holds.
+    """
+    c = cfg.c()
+    _check("lazy_decode_attn_noalloc", _lib.lazy_decode_attn_noalloc(
+        ctypes.byref(c), _ptr(q_raw), _ptr(q_pos), int(q_pos.numel()), _ptr(table), _ptr(table_indptr),
+        int(max_words), _ptr(blk_meta), _ptr(k_pool), _ptr(v_pool), int(k_pool.shape[0]), _ptr(out),
+        _ptr(d_status), _stream(stream)))
