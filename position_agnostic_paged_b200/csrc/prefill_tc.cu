@@ -1,37 +1,42 @@
 // prefill_tc.cu -- causal prefill attention over the paged pool with deferred
 // RoPE on the fifth-generation tensor cores (tcgen05.mma, accumulators in
-// tensor memory, operands staged by TMA).
+// tensor memory, K/V tiles staged by TMA).
 //
 // Source: gist.science, "LazyAttention: Efficient Retrieval-Augmented
 // Generation with Deferred Positional Encoding", Technical Summary, Technical
 // Implementation: Prefilling -- the kernel loads cached KV blocks and applies
 // one relative rotation based on the offset between the query and the cached
 // document instead of resetting the keys to position 0 and rotating them
-// again; the attention is compute-bound.
+// again; this phase is compute-bound.
 //
 // Where the single relative rotation goes.  Keys sit in the pool rotated at
-// their local index j.  For a query tile whose first token is at position P,
-// the rotation warpgroup keeps Qt = R(p_i - P) q_i (once per CTA, bf16 in
-// shared memory).  Each time the table walk enters a segment with offset o it
-// writes Q' = R(P - o) Qt into one of two query buffers: one relative
-// rotation by (P - o), uniform across the tile, so scores carry the angle
-// (p_i - o - j) of eager RoPE attention.  Stored keys go from TMA to the
-// tensor core untouched, and the rotation overlaps the MMAs of the previous
-// segment.
+// their local index j.  For every segment (document) that the table walk
+// enters, with logical offset o, the rotation warpgroup writes the query tile
+// Q'_i = R(p_i - o) q_i once; stored keys go from TMA to the tensor core
+// untouched and scores carry the angle (p_i - o - j) of eager RoPE attention.
+// The rewrite of the query tile overlaps the softmax of the segment's last
+// key tile, so it costs no tensor-core time.
 //
-// CTA = one 128-row query tile (rows are (token, head-in-group) pairs,
-// token-major) of one KV head of one request; 12 warps:
-//   warp 0       TMA producer: per KV tile (<= 8 blocks = 128 keys of one
-//                segment) the K and V boxes into double-buffered stages
-//   warp 1       tensor-memory owner and MMA issuer: S = Q' K^T (8 MMAs,
-//                K = 16 each) into S[j%2], then O += P V (one MMA per block)
-//   warps 2-3    idle
-//   warps 4-7    softmax, one thread per query row: S row from tensor memory,
-//                mask, online softmax with lazy rescaling of O, P (bf16) back
-//                to tensor memory; the epilogue writes O / l
-//   warps 8-11   query rotation (Qt once, then Q' per segment)
-// Tensor memory (512 columns): S0 [0,128) S1 [128,256) O [256,384)
-// P0 [384,448) P1 [448,512).
+// CTA = 256 query rows (two 128-row MMA tiles) of one KV head of one
+// request; rows are (token, head-in-group) pairs, token-major, so each K/V
+// tile loaded by TMA serves every query head of its group and both row
+// tiles.  16 warps:
+//   warp 0      K producer: walks the table once, publishes per-tile
+//               information (blocks, metadata, mask flags, segment flags) in
+//               a shared-memory ring, and TMA-loads K tiles (<= 8 blocks =
+//               128 keys of one segment) into 3 stages
+//   warp 1      V producer: TMA-loads V tiles into 2 stages
+//   warp 2      tensor-memory owner and MMA issuer, in the order
+//               QK0(j), PV1(j-1), QK1(j), PV0(j): while one softmax
+//               warpgroup works on its tile the tensor core runs the other's
+//   warp 3      idle
+//   warps 4-7   softmax of row tile 0, one thread per row: S from tensor
+//               memory, mask, online softmax with lazy rescaling of O, P
+//               (bf16) written over the consumed S columns; epilogue O / l
+//   warps 8-11  softmax of row tile 1
+//   warps 12-15 query rotation, once per segment
+// Tensor memory (512 columns): S0 [0,128) (P0 = its first 64 columns),
+// S1 [128,256) (P1), O0 [256,384), O1 [384,512).
 #include <climits>
 
 #include "common.cuh"
@@ -42,47 +47,48 @@ namespace lazy {
 
 namespace {
 
-constexpr int kRows = 128;
+constexpr int kTileRows = 128;
+constexpr int kRows = 2 * kTileRows;
 constexpr int kTileBlocks = 8;
-constexpr int kTileBytes = kRows * kHeadDim * 2;   // 32 KiB
-constexpr int kHalfPlane = kTileBytes / 2;         // 16 KiB
-constexpr int kThreads = 384;
+constexpr int kTileBytes = kTileRows * kHeadDim * 2;   // 32 KiB
+constexpr int kHalfPlane = kTileBytes / 2;             // 16 KiB
+constexpr int kKStages = 3, kVStages = 2, kInfoStages = 8;
+constexpr int kThreads = 512;
 
-constexpr int kOffQt = 0;
-constexpr int kOffQ = kOffQt + kTileBytes;
-constexpr int kOffK = kOffQ + 2 * kTileBytes;
-constexpr int kOffV = kOffK + 2 * kTileBytes;
-constexpr int kOffBar = kOffV + 2 * kTileBytes;
-constexpr int kNumBars = 21;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kOffSeg = kOffMisc + 16;
-constexpr int kOffTheta = kOffSeg + kHalfDim * 8;
-constexpr int kSmemUse = kOffTheta + kHalfDim * 8;
+struct TileInfo {
+    uint32_t blk[kTileBlocks];
+    uint32_t meta[kTileBlocks];
+    int n;       // blocks in the tile (1..8)
+    int off;     // the segment's logical offset
+    int flags;   // kFull | kNewSeg | kSegEnd
+    int pad;
+};
+constexpr int kFull = 1, kNewSeg = 2, kSegEnd = 4;
+
+constexpr int kOffQ = 0;                                     // 2 row tiles
+constexpr int kOffK = kOffQ + 2 * kTileBytes;                // 3 stages
+constexpr int kOffV = kOffK + kKStages * kTileBytes;         // 2 stages
+constexpr int kOffInfo = kOffV + kVStages * kTileBytes;
+constexpr int kOffBar = kOffInfo + kInfoStages * static_cast<int>(sizeof(TileInfo));
+// barriers
+constexpr int B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_VFULL = B_KEMPTY + kKStages,
+              B_VEMPTY = B_VFULL + kVStages, B_IFULL = B_VEMPTY + kVStages, B_IEMPTY = B_IFULL + kInfoStages,
+              B_SFULL = B_IEMPTY + kInfoStages, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2, B_QFULL = B_ODONE + 2,
+              B_QEMPTY = B_QFULL + 1, B_DRAIN = B_QEMPTY + 1, kNumBars = B_DRAIN + 1;
+constexpr int kOffTheta = kOffBar + kNumBars * 8;
+constexpr int kOffSeg = kOffTheta + kHalfDim * 8;
+constexpr int kOffMisc = kOffSeg + kHalfDim * 8;
+constexpr int kSmemUse = kOffMisc + 16;
 constexpr size_t kTcSmem = kSmemUse + 1024;
 static_assert(kTcSmem <= 232448, "shared memory budget");
-
-// barrier indices
-constexpr int B_KFULL = 0, B_KEMPTY = 2, B_VFULL = 4, B_VEMPTY = 6, B_SFULL = 8, B_SFREE = 10, B_PFULL = 12,
-              B_ODONE = 14, B_QFULL = 16, B_QEMPTY = 18, B_DRAIN = 20;
+static_assert(sizeof(TileInfo) == 80, "tile info layout");
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays below 2^8 between rescales
+// consumers of one tile-info entry: 8 softmax warps, the V producer, the MMA issuer
+constexpr int kInfoConsumers = 10;
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-struct KTile {
-    int n;     // blocks in the tile (1..8), all from one segment
-    int off;   // the segment's logical offset
-};
-
-// Tiles are formed identically by every role: up to 8 consecutive table words
-// that share one offset (a tile never spans two segments).
-__device__ __forceinline__ KTile ktile(const uint32_t *tbl, int w, int n_words) {
-    const int off = word_offset(tbl[w]);
-    int n = 1;
-    while (n < kTileBlocks && w + n < n_words && word_offset(tbl[w + n]) == off) ++n;
-    return {n, off};
 }
 
 // Bounded wait that also gives up as soon as another role has aborted.
@@ -96,16 +102,13 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
     set_status(d_status, LAZY_DSTATUS_TIMEOUT);
     return false;
 }
-
-__device__ __forceinline__ void rot_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
-
-// Same decision for every lane of the warp (a lane whose poll ran out aborts all).
+// Same decision for every lane of the warp.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *d_status) {
     const bool ok = wait_or_abort(bar, parity, abort_flag, d_status);
     return __all_sync(0xffffffffu, ok);
 }
-
-// Same decision for the 128 threads of the rotation warpgroup (named barrier 2).
+__device__ __forceinline__ void rot_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+// Same decision for the 128 threads of the rotation warpgroup.
 __device__ __forceinline__ bool rot_all(bool ok) {
     uint32_t any_fail;
     asm volatile(
@@ -124,10 +127,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
+    TileInfo *info = reinterpret_cast<TileInfo *>(sm + kOffInfo);
+    double *theta_s = reinterpret_cast<double *>(sm + kOffTheta);
+    float2 *segcs = reinterpret_cast<float2 *>(sm + kOffSeg);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);
-    float2 *segcs = reinterpret_cast<float2 *>(sm + kOffSeg);
-    double *theta_s = reinterpret_cast<double *>(sm + kOffTheta);
 
     const int mt = blockIdx.x, kvh = blockIdx.y, r = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -140,37 +144,37 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     const int n_words = p.table_indptr[r + 1] - wbase;
     const uint32_t *tbl = p.table + wbase;
     const int pos0 = p.q_pos0[r];
-    const int tok_base = R0 / G;
-    const int Pbase = pos0 + tok_base;
+    const int tok_first = R0 / G;
+    const int tok_last = min(T - 1, (R0 + kRows - 1) / G);
+    const int Pbase = pos0 + tok_first;   // smallest query position of the CTA
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars[B_KFULL], 1);
-        mbar_init(&bars[B_KFULL + 1], 1);
-        mbar_init(&bars[B_KEMPTY], 1);
-        mbar_init(&bars[B_KEMPTY + 1], 1);
-        mbar_init(&bars[B_VFULL], 1);
-        mbar_init(&bars[B_VFULL + 1], 1);
-        mbar_init(&bars[B_VEMPTY], 1);
-        mbar_init(&bars[B_VEMPTY + 1], 1);
-        mbar_init(&bars[B_SFULL], 1);
-        mbar_init(&bars[B_SFULL + 1], 1);
-        mbar_init(&bars[B_SFREE], 4);
-        mbar_init(&bars[B_SFREE + 1], 4);
-        mbar_init(&bars[B_PFULL], 4);
-        mbar_init(&bars[B_PFULL + 1], 4);
-        mbar_init(&bars[B_ODONE], 1);
-        mbar_init(&bars[B_ODONE + 1], 1);
+        for (int i = 0; i < kKStages; ++i) {
+            mbar_init(&bars[B_KFULL + i], 1);
+            mbar_init(&bars[B_KEMPTY + i], 1);
+        }
+        for (int i = 0; i < kVStages; ++i) {
+            mbar_init(&bars[B_VFULL + i], 1);
+            mbar_init(&bars[B_VEMPTY + i], 1);
+        }
+        for (int i = 0; i < kInfoStages; ++i) {
+            mbar_init(&bars[B_IFULL + i], 1);
+            mbar_init(&bars[B_IEMPTY + i], kInfoConsumers);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bars[B_SFULL + t], 1);
+            mbar_init(&bars[B_PFULL + t], 4);
+            mbar_init(&bars[B_ODONE + t], 1);
+        }
         mbar_init(&bars[B_QFULL], 4);
-        mbar_init(&bars[B_QFULL + 1], 4);
         mbar_init(&bars[B_QEMPTY], 1);
-        mbar_init(&bars[B_QEMPTY + 1], 1);
         mbar_init(&bars[B_DRAIN], 1);
         *abort_flag = 0;
         if (mt == 0 && kvh == 0 && n_words > p.max_words) set_status(p.d_status, LAZY_DSTATUS_BAD_TABLE);
         fence_barrier_init();
     }
     if (threadIdx.x < kHalfDim) theta_s[threadIdx.x] = p.rope.theta[threadIdx.x];
-    if (warp == 1) {
+    if (warp == 2) {
         tc::tmem_alloc(tmem_slot, 512);
         tc::tmem_relinquish();
     }
@@ -178,157 +182,211 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tbase = *tmem_slot;
-    const uint32_t tS0 = tbase, tO = tbase + 256, tP0 = tbase + 384;
 
     if (warp == 0) {
-        // ============================================================ TMA producer
+        // ============================================================ table walk + K producer
         if (lane == 0) {
             tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            int issued = 0;
+            int issued = 0, prev_off = INT_MIN;
             for (int w = 0, j = 0; w < n_words; ++j) {
-                const KTile t = ktile(tbl, w, n_words);
-                const int st = j & 1;
-                const uint32_t ph = ((j >> 1) & 1) ^ 1;
-                if (!wait_or_abort(&bars[B_KEMPTY + st], ph, abort_flag, p.d_status)) break;
-                mbar_arrive_expect_tx(&bars[B_KFULL + st], t.n * kBlockBytes);
-                uint8_t *kd = sm + kOffK + st * kTileBytes;
-                for (int k = 0; k < t.n; ++k) {
-                    const uint32_t b = word_block(tbl[w + k]);
+                // the tile: up to 8 consecutive words that share one offset
+                uint32_t wd[kTileBlocks];
+#pragma unroll
+                for (int k = 0; k < kTileBlocks; ++k) wd[k] = (w + k < n_words) ? tbl[w + k] : 0xFFFFFFFFu;
+                const int off = word_offset(wd[0]);
+                int n = 1;
+#pragma unroll
+                for (int k = 1; k < kTileBlocks; ++k)
+                    if (n == k && w + k < n_words && word_offset(wd[k]) == off) n = k + 1;
+                const int wn = w + n;
+                const int off_rot = PLAIN ? 0 : off;
+                const int next_rot = wn < n_words ? (PLAIN ? 0 : word_offset(tbl[wn])) : INT_MIN;
+                uint32_t mt_k[kTileBlocks];
+                bool full = n == kTileBlocks;
+#pragma unroll
+                for (int k = 0; k < kTileBlocks; ++k) {
+                    const uint32_t b = word_block(wd[k]);
+                    const bool ok = k < n && b < static_cast<uint32_t>(p.num_blocks);
+                    mt_k[k] = ok ? p.blk_meta[b] : 0u;
+                    if (k < n && !ok) set_status(p.d_status, LAZY_DSTATUS_BAD_BLOCK);
+                    full = full && meta_valid(mt_k[k]) == kBlockTokens &&
+                           off + meta_j0(mt_k[k]) + kBlockTokens - 1 <= Pbase;
+                }
+                const int flags = (full ? kFull : 0) | (off_rot != prev_off ? kNewSeg : 0) |
+                                  (next_rot != off_rot ? kSegEnd : 0);
+                prev_off = off_rot;
+                // publish the tile information
+                const int is = j % kInfoStages;
+                if (!wait_or_abort(&bars[B_IEMPTY + is], ((j / kInfoStages) & 1) ^ 1, abort_flag, p.d_status)) break;
+                TileInfo &ti = info[is];
+#pragma unroll
+                for (int k = 0; k < kTileBlocks; ++k) {
+                    ti.blk[k] = k < n ? word_block(wd[k]) : 0u;
+                    ti.meta[k] = mt_k[k];
+                }
+                ti.n = n;
+                ti.off = off;
+                ti.flags = flags;
+                mbar_arrive(&bars[B_IFULL + is]);
+                // K tile
+                const int ks = j % kKStages;
+                if (!wait_or_abort(&bars[B_KEMPTY + ks], ((j / kKStages) & 1) ^ 1, abort_flag, p.d_status)) break;
+                mbar_arrive_expect_tx(&bars[B_KFULL + ks], n * kBlockBytes);
+                uint8_t *kd = sm + kOffK + ks * kTileBytes;
+                for (int k = 0; k < n; ++k) {
+                    const uint32_t b = word_block(wd[k]);
                     int row;
                     if (b >= static_cast<uint32_t>(p.num_blocks)) {
-                        set_status(p.d_status, LAZY_DSTATUS_BAD_BLOCK);
                         row = p.k_rows;   // fully out of bounds: the box is zero-filled
                     } else {
                         row = PLAIN ? ((wbase + w + k) * p.hkv + kvh) * kBlockTokens
                                     : (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens;
                     }
-                    tma_load_2d(kd + k * kBoxBytes, &tmK, 0, row, &bars[B_KFULL + st]);
-                    tma_load_2d(kd + kHalfPlane + k * kBoxBytes, &tmK, kHalfDim, row, &bars[B_KFULL + st]);
-                }
-                if (!wait_or_abort(&bars[B_VEMPTY + st], ph, abort_flag, p.d_status)) {
-                    issued = j + 1;   // K of this tile is in flight
-                    break;
-                }
-                mbar_arrive_expect_tx(&bars[B_VFULL + st], t.n * kBlockBytes);
-                uint8_t *vd = sm + kOffV + st * kTileBytes;
-                for (int k = 0; k < t.n; ++k) {
-                    const uint32_t b = word_block(tbl[w + k]);
-                    const int row = b >= static_cast<uint32_t>(p.num_blocks)
-                                        ? p.v_rows
-                                        : (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens;
-                    tma_load_2d(vd + k * kBoxBytes, &tmV, 0, row, &bars[B_VFULL + st]);
-                    tma_load_2d(vd + kHalfPlane + k * kBoxBytes, &tmV, kHalfDim, row, &bars[B_VFULL + st]);
+                    tma_load_2d(kd + k * kBoxBytes, &tmK, 0, row, &bars[B_KFULL + ks]);
+                    tma_load_2d(kd + kHalfPlane + k * kBoxBytes, &tmK, kHalfDim, row, &bars[B_KFULL + ks]);
                 }
                 issued = j + 1;
-                w += t.n;
+                w = wn;
             }
-            // no copy may land after the CTA exits: wait for the last phase of each armed stage
-            for (int j = max(0, issued - 2); j < issued; ++j) {
-                mbar_wait(&bars[B_KFULL + (j & 1)], (j >> 1) & 1);
-                mbar_wait(&bars[B_VFULL + (j & 1)], (j >> 1) & 1);
-            }
+            for (int j = max(0, issued - kKStages); j < issued; ++j)
+                mbar_wait(&bars[B_KFULL + j % kKStages], (j / kKStages) & 1);
         }
     } else if (warp == 1) {
+        // ============================================================ V producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmV);
+            int issued = 0;
+            for (int w = 0, j = 0; w < n_words; ++j) {
+                const int is = j % kInfoStages;
+                if (!wait_or_abort(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) break;
+                const int n = info[is].n;
+                uint32_t blk[kTileBlocks];
+#pragma unroll
+                for (int k = 0; k < kTileBlocks; ++k) blk[k] = info[is].blk[k];
+                mbar_arrive(&bars[B_IEMPTY + is]);
+                const int vs = j % kVStages;
+                if (!wait_or_abort(&bars[B_VEMPTY + vs], ((j / kVStages) & 1) ^ 1, abort_flag, p.d_status)) break;
+                mbar_arrive_expect_tx(&bars[B_VFULL + vs], n * kBlockBytes);
+                uint8_t *vd = sm + kOffV + vs * kTileBytes;
+                for (int k = 0; k < n; ++k) {
+                    const int row = blk[k] >= static_cast<uint32_t>(p.num_blocks)
+                                        ? p.v_rows
+                                        : (static_cast<int>(blk[k]) * p.hkv + kvh) * kBlockTokens;
+                    tma_load_2d(vd + k * kBoxBytes, &tmV, 0, row, &bars[B_VFULL + vs]);
+                    tma_load_2d(vd + kHalfPlane + k * kBoxBytes, &tmV, kHalfDim, row, &bars[B_VFULL + vs]);
+                }
+                issued = j + 1;
+                w += n;
+            }
+            for (int j = max(0, issued - kVStages); j < issued; ++j)
+                mbar_wait(&bars[B_VFULL + j % kVStages], (j / kVStages) & 1);
+        }
+    } else if (warp == 2) {
         // ============================================================ MMA issuer
         if (lane == 0) {
             const uint32_t idq = tc::idesc_bf16(128, 128, false);
             const uint32_t idv = tc::idesc_bf16(128, 128, true);
             const uint32_t sQ = smem_u32(sm + kOffQ), sK = smem_u32(sm + kOffK), sV = smem_u32(sm + kOffV);
-            int seg = -1, cur = INT_MIN, prev_n = 0, j = 0;
+            const uint32_t tS[2] = {tbase, tbase + 128}, tO[2] = {tbase + 256, tbase + 384};
+            int seg = 0, prev_n = 0, j = 0;
             bool ok = true;
-            auto issue_pv = [&](int t, int n) -> bool {
-                const int s = t & 1;
-                if (!wait_or_abort(&bars[B_VFULL + s], (t >> 1) & 1, abort_flag, p.d_status)) return false;
-                if (!wait_or_abort(&bars[B_PFULL + s], (t >> 1) & 1, abort_flag, p.d_status)) return false;
-                tc::fence_after_sync();
-                const uint32_t vb = sV + s * kTileBytes;
-                for (int k = 0; k < n; ++k)
-                    tc::mma_ts(tO, tP0 + 64 * s + 8 * k, tc::smem_desc(vb + k * kBoxBytes, kHalfPlane, 1024), idv,
-                               (t > 0 || k > 0) ? 1u : 0u);
-                tc::commit(&bars[B_ODONE + s]);
-                tc::commit(&bars[B_VEMPTY + s]);
-                return true;
-            };
-            for (int w = 0; w < n_words && ok; ++j) {
-                const KTile t = ktile(tbl, w, n_words);
-                const int off_rot = PLAIN ? 0 : t.off;
-                if (off_rot != cur) {
-                    ++seg;
-                    cur = off_rot;
-                    if (!wait_or_abort(&bars[B_QFULL + (seg & 1)], (seg >> 1) & 1, abort_flag, p.d_status)) break;
-                }
-                const int s = j & 1;
-                if (!wait_or_abort(&bars[B_KFULL + s], (j >> 1) & 1, abort_flag, p.d_status)) break;
-                if (j >= 2 && !wait_or_abort(&bars[B_SFREE + s], ((j - 2) >> 1) & 1, abort_flag, p.d_status)) break;
-                tc::fence_after_sync();
-                const uint32_t qa = sQ + (seg & 1) * kTileBytes, kb = sK + s * kTileBytes;
+            auto qk = [&](int t, int ks) {
+                const uint32_t qa = sQ + t * kTileBytes, kb = sK + ks * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t o = (kk >> 2) * kHalfPlane + (kk & 3) * 32;
-                    tc::mma_ss(tS0 + 128 * s, tc::smem_desc(qa + o, 16, 1024), tc::smem_desc(kb + o, 16, 1024), idq,
+                    tc::mma_ss(tS[t], tc::smem_desc(qa + o, 16, 1024), tc::smem_desc(kb + o, 16, 1024), idq,
                                kk > 0 ? 1u : 0u);
                 }
-                tc::commit(&bars[B_SFULL + s]);
-                tc::commit(&bars[B_KEMPTY + s]);
-                const int wn = w + t.n;
-                const bool seg_end = wn >= n_words || (PLAIN ? false : word_offset(tbl[wn]) != off_rot);
-                if (seg_end) tc::commit(&bars[B_QEMPTY + (seg & 1)]);
-                if (j >= 1) ok = issue_pv(j - 1, prev_n);
-                prev_n = t.n;
-                w = wn;
+                tc::commit(&bars[B_SFULL + t]);
+            };
+            // O_t += P_t V(jj); P_t occupies the first 64 columns of S_t
+            auto pv = [&](int t, int jj, int n) -> bool {
+                const int vs = jj % kVStages;
+                if (!wait_or_abort(&bars[B_VFULL + vs], (jj / kVStages) & 1, abort_flag, p.d_status)) return false;
+                if (!wait_or_abort(&bars[B_PFULL + t], jj & 1, abort_flag, p.d_status)) return false;
+                tc::fence_after_sync();
+                const uint32_t vb = sV + vs * kTileBytes;
+                for (int k = 0; k < n; ++k)
+                    tc::mma_ts(tO[t], tS[t] + 8 * k, tc::smem_desc(vb + k * kBoxBytes, kHalfPlane, 1024), idv,
+                               (jj > 0 || k > 0) ? 1u : 0u);
+                tc::commit(&bars[B_ODONE + t]);
+                if (t == 1) tc::commit(&bars[B_VEMPTY + vs]);   // V(jj) fully consumed
+                return true;
+            };
+            for (int w = 0; w < n_words && ok; ++j) {
+                const int is = j % kInfoStages;
+                if (!wait_or_abort(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) break;
+                const int n = info[is].n, flags = info[is].flags;
+                mbar_arrive(&bars[B_IEMPTY + is]);
+                if (flags & kNewSeg) {
+                    if (!wait_or_abort(&bars[B_QFULL], seg & 1, abort_flag, p.d_status)) break;
+                    ++seg;
+                }
+                const int ks = j % kKStages;
+                if (!wait_or_abort(&bars[B_KFULL + ks], (j / kKStages) & 1, abort_flag, p.d_status)) break;
+                tc::fence_after_sync();
+                qk(0, ks);
+                if (j >= 1 && !(ok = pv(1, j - 1, prev_n))) break;
+                qk(1, ks);
+                tc::commit(&bars[B_KEMPTY + ks]);
+                if (flags & kSegEnd) tc::commit(&bars[B_QEMPTY]);
+                if (!(ok = pv(0, j, n))) break;
+                prev_n = n;
+                w += n;
             }
-            if (ok && j >= 1 && !*abort_flag) issue_pv(j - 1, prev_n);
+            if (ok && j >= 1 && !*abort_flag) pv(1, j - 1, prev_n);
             // every MMA this thread issued has completed before tensor memory is freed
             tc::commit(&bars[B_DRAIN]);
             mbar_wait(&bars[B_DRAIN], 0);
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 4 && warp < 12) {
         // ============================================================ softmax (one row per thread)
-        const int row = threadIdx.x - 128;
-        const int R = R0 + row;
+        const int t = (warp - 4) >> 2;                 // row tile
+        const int row = threadIdx.x - 128 - 128 * t;   // 0..127 inside the tile
+        const int R = R0 + kTileRows * t + row;
         const bool row_ok = R < T * G;
-        const int tok = row_ok ? R / G : tok_base;
+        const int tok = row_ok ? R / G : tok_first;
         const int g = R % G;
         const int prow = pos0 + tok;
-        const uint32_t lane_off = static_cast<uint32_t>(32 * (warp - 4)) << 16;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+        const uint32_t tS = tbase + 128 * t, tO = tbase + 256 + 128 * t;
         float m_run = -INFINITY, l_run = 0.f;
         int j = 0;
         bool ok = true;
         for (int w = 0; w < n_words; ++j) {
-            const KTile t = ktile(tbl, w, n_words);
-            const int s = j & 1;
-            if (!warp_wait(&bars[B_SFULL + s], (j >> 1) & 1, abort_flag, p.d_status)) { ok = false; break; }
-            tc::fence_after_sync();
-            // block metadata of the tile (positions for the causal mask, valid slots)
+            const int is = j % kInfoStages;
+            if (!warp_wait(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) { ok = false; break; }
+            const TileInfo &ti = info[is];
+            const int n = ti.n, off = ti.off;
+            const bool full = (ti.flags & kFull) != 0;
             int kj0[kTileBlocks], knv[kTileBlocks];
-            bool full = t.n == kTileBlocks;
 #pragma unroll
             for (int k = 0; k < kTileBlocks; ++k) {
-                kj0[k] = 0;
-                knv[k] = 0;
-                if (k < t.n) {
-                    const uint32_t b = word_block(tbl[w + k]);
-                    if (b < static_cast<uint32_t>(p.num_blocks)) {
-                        const uint32_t mm = p.blk_meta[b];
-                        kj0[k] = meta_j0(mm);
-                        knv[k] = meta_valid(mm);
-                    }
-                }
-                full = full && knv[k] == kBlockTokens && t.off + kj0[k] + kBlockTokens - 1 <= Pbase;
+                kj0[k] = meta_j0(ti.meta[k]);
+                knv[k] = k < n ? meta_valid(ti.meta[k]) : 0;
             }
-            // pass 1 over the S row in tensor memory: masked row maximum
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[B_IEMPTY + is]);
+            if (!warp_wait(&bars[B_SFULL + t], j & 1, abort_flag, p.d_status)) { ok = false; break; }
+            tc::fence_after_sync();
+            // pass 1: masked row maximum (S_t(j) complete implies PV_t(j-1) complete)
             float tmax = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t x[32];
-                tc::ld32(tS0 + 128 * s + lane_off + 32 * c, x);
+                tc::ld32(tS + lane_off + 32 * c, x);
                 tc::wait_ld();
+                if (full) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int col = 32 * c + e, k = col >> 4, si = col & 15;
-                    const bool vis = full || (si < knv[k] && t.off + kj0[k] + si <= prow);
-                    tmax = vis ? fmaxf(tmax, __uint_as_float(x[e])) : tmax;
+                    for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, __uint_as_float(x[e]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int col = 32 * c + e, k = col >> 4, si = col & 15;
+                        const bool vis = si < knv[k] && off + kj0[k] + si <= prow;
+                        tmax = vis ? fmaxf(tmax, __uint_as_float(x[e])) : tmax;
+                    }
                 }
             }
             const float m_new = fmaxf(m_run, tmax);
@@ -340,12 +398,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 l_run *= scale;
             }
             if (j > 0 && __any_sync(0xffffffffu, need)) {
-                // O must be complete up to tile j-1 before it is rescaled in place
-                if (!warp_wait(&bars[B_ODONE + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort_flag, p.d_status)) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t o[32];
@@ -355,21 +407,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * scale);
                     tc::st32(tO + lane_off + 32 * c, o);
                 }
-                tc::wait_st();
             }
             const float mu = m_run == -INFINITY ? 0.f : m_run;
-            // P[j%2] is free once the PV product of tile j-2 has completed
-            if (j >= 2 && !warp_wait(&bars[B_ODONE + s], ((j - 2) >> 1) & 1, abort_flag, p.d_status)) {
-                ok = false;
-                break;
-            }
-            tc::fence_after_sync();
-            // pass 2: P = 2^(S - m) as bf16 pairs into tensor memory, row sum in fp32
+            // pass 2: P = 2^(S - m) as bf16 pairs over the consumed S columns, row sum in fp32
             float lsum = 0.f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t x[32], pk[16];
-                tc::ld32(tS0 + 128 * s + lane_off + 32 * c, x);
+                tc::ld32(tS + lane_off + 32 * c, x);
                 tc::wait_ld();
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -377,154 +422,136 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int col = 32 * c + 2 * e + h, k = col >> 4, si = col & 15;
-                        const bool vis = full || (si < knv[k] && t.off + kj0[k] + si <= prow);
+                        const bool vis = full || (si < knv[k] && off + kj0[k] + si <= prow);
                         pr[h] = vis ? fast_exp2(__uint_as_float(x[2 * e + h]) - mu) : 0.f;
                     }
                     lsum += pr[0] + pr[1];
                     pk[e] = pack_bf16(pr[0], pr[1]);
                 }
-                tc::st16(tP0 + 64 * s + lane_off + 16 * c, pk);
+                tc::st16(tS + lane_off + 16 * c, pk);   // columns already read in this or an earlier chunk
             }
             l_run += lsum;
             tc::wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bars[B_SFREE + s]);
-                mbar_arrive(&bars[B_PFULL + s]);
-            }
-            w += t.n;
+            if (lane == 0) mbar_arrive(&bars[B_PFULL + t]);
+            w += n;
         }
         // ------------------------------------------------------------ epilogue
-        uint32_t ob[4][32];
         bool have = ok && j > 0;
-        if (have) {
-            have = warp_wait(&bars[B_ODONE + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort_flag, p.d_status);
-        }
+        if (have) have = warp_wait(&bars[B_ODONE + t], (j - 1) & 1, abort_flag, p.d_status);
         const float inv = (have && l_run > 0.f) ? 1.f / l_run : 0.f;
-        if (__all_sync(0xffffffffu, have)) {
-            tc::fence_after_sync();
+        const bool all_have = __all_sync(0xffffffffu, have);
+        if (all_have) tc::fence_after_sync();
+        uint4 *o = row_ok ? reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(q0 + tok) * p.hq + kvh * G + g) *
+                                                                  kHeadDim)
+                          : nullptr;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tc::ld32(tO + lane_off + 32 * c, ob[c]);
-            tc::wait_ld();
-        } else {
+        for (int c = 0; c < 4; ++c) {
+            uint32_t ob[32];
+            if (all_have) {
+                tc::ld32(tO + lane_off + 32 * c, ob);
+                tc::wait_ld();
+            } else {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int e = 0; e < 32; ++e) ob[c][e] = 0u;
-        }
-        if (row_ok) {
-            uint4 *o = reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(q0 + tok) * p.hq + kvh * G + g) *
-                                                             kHeadDim);
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
+                for (int e = 0; e < 32; ++e) ob[e] = 0u;
+            }
+            if (o) {
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                     uint4 u;
-                    u.x = pack_bf16(__uint_as_float(ob[c][8 * v + 0]) * inv, __uint_as_float(ob[c][8 * v + 1]) * inv);
-                    u.y = pack_bf16(__uint_as_float(ob[c][8 * v + 2]) * inv, __uint_as_float(ob[c][8 * v + 3]) * inv);
-                    u.z = pack_bf16(__uint_as_float(ob[c][8 * v + 4]) * inv, __uint_as_float(ob[c][8 * v + 5]) * inv);
-                    u.w = pack_bf16(__uint_as_float(ob[c][8 * v + 6]) * inv, __uint_as_float(ob[c][8 * v + 7]) * inv);
+                    u.x = pack_bf16(__uint_as_float(ob[8 * v + 0]) * inv, __uint_as_float(ob[8 * v + 1]) * inv);
+                    u.y = pack_bf16(__uint_as_float(ob[8 * v + 2]) * inv, __uint_as_float(ob[8 * v + 3]) * inv);
+                    u.z = pack_bf16(__uint_as_float(ob[8 * v + 4]) * inv, __uint_as_float(ob[8 * v + 5]) * inv);
+                    u.w = pack_bf16(__uint_as_float(ob[8 * v + 6]) * inv, __uint_as_float(ob[8 * v + 7]) * inv);
                     o[4 * c + v] = u;
                 }
-        }
-    } else if (warp >= 8) {
-        // ============================================================ query rotation
-        const int tid = threadIdx.x - 256;
-        const int ch = tid & 7;          // 8-pair chunk: pairs 8ch .. 8ch+7
-        const int rbase = tid >> 3;      // rows rbase + 16k
-        uint8_t *qt = sm + kOffQt;
-        // Qt = R(p_i - P) q_i, pre-scaled by softmax_scale * log2(e)
-#pragma unroll 1
-        for (int k = 0; k < 8; ++k) {
-            const int rr = rbase + 16 * k;
-            const int Rr = R0 + rr;
-            uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
-            if (Rr < T * G) {
-                const int tk = Rr / G, gg = Rr % G;
-                const uint16_t *q = p.q_raw + (static_cast<size_t>(q0 + tk) * p.hq + kvh * G + gg) * kHeadDim;
-                const uint4 a4 = *reinterpret_cast<const uint4 *>(q + 8 * ch);
-                const uint4 b4 = *reinterpret_cast<const uint4 *>(q + kHalfDim + 8 * ch);
-                const uint32_t *aw = reinterpret_cast<const uint32_t *>(&a4);
-                const uint32_t *bw = reinterpret_cast<const uint32_t *>(&b4);
-                uint32_t *lw = reinterpret_cast<uint32_t *>(&lo);
-                uint32_t *hw = reinterpret_cast<uint32_t *>(&hi);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float c0, s0, c1, s1;
-                    rope_cos_sin(tk - tok_base, theta_s[8 * ch + 2 * e], c0, s0);
-                    rope_cos_sin(tk - tok_base, theta_s[8 * ch + 2 * e + 1], c1, s1);
-                    const float a0 = bf16_lo(aw[e]) * p.scale_log2, a1 = bf16_hi(aw[e]) * p.scale_log2;
-                    const float b0 = bf16_lo(bw[e]) * p.scale_log2, b1 = bf16_hi(bw[e]) * p.scale_log2;
-                    lw[e] = pack_bf16(a0 * c0 - b0 * s0, a1 * c1 - b1 * s1);
-                    hw[e] = pack_bf16(b0 * c0 + a0 * s0, b1 * c1 + a1 * s1);
-                }
             }
-            const uint32_t off = rr * 128 + ((ch ^ (rr & 7)) << 4);
-            *reinterpret_cast<uint4 *>(qt + off) = lo;
-            *reinterpret_cast<uint4 *>(qt + kHalfPlane + off) = hi;
         }
-        rot_sync();
-        int seg = -1, cur = INT_MIN;
-        for (int w = 0; w < n_words;) {
-            const KTile t = ktile(tbl, w, n_words);
-            w += t.n;
-            const int off_rot = PLAIN ? 0 : t.off;
+    } else if (warp >= 12) {
+        // ============================================================ query rotation
+        const int tid = threadIdx.x - 384;
+        const int ch = tid & 7;         // pairs 8ch .. 8ch+7
+        const int tl = tid >> 3;        // tokens tok_first + tl + 16k
+        // per-thread constants: rotation by 16 tokens, and by (tl tokens) from the CTA's first token
+        float c16[8], s16[8], cb[8], sb[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            rope_cos_sin(16, theta_s[8 * ch + e], c16[e], s16[e]);
+            rope_cos_sin(tl, theta_s[8 * ch + e], cb[e], sb[e]);
+        }
+        int seg = 0, cur = INT_MIN;
+        for (int w = 0; w < n_words; ++w) {
+            const int off_rot = PLAIN ? 0 : word_offset(tbl[w]);
             if (off_rot == cur) continue;
-            ++seg;
             cur = off_rot;
-            const int qb = seg & 1;
-            bool ok = true;
-            if (seg >= 2) ok = wait_or_abort(&bars[B_QEMPTY + qb], ((seg - 2) >> 1) & 1, abort_flag, p.d_status);
-            if (!rot_all(ok)) break;
-            // the segment's uniform rotation R(P - o), one pair per thread
+            bool okw = true;
+            if (seg >= 1) okw = wait_or_abort(&bars[B_QEMPTY], (seg - 1) & 1, abort_flag, p.d_status);
+            if (!rot_all(okw)) break;
+            // the segment's rotation R(P - o), one pair per thread
             if (tid < kHalfDim) {
                 float c, s;
                 rope_cos_sin(Pbase - off_rot, theta_s[tid], c, s);
                 segcs[tid] = make_float2(c, s);
             }
             rot_sync();
-            float cs[8], sn[8];
+            // angle of this thread's first token: R(P - o) composed with R(tl)
+            float cc[8], ss[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const float2 v = segcs[8 * ch + e];
-                cs[e] = v.x;
-                sn[e] = v.y;
+                cc[e] = v.x * cb[e] - v.y * sb[e];
+                ss[e] = v.y * cb[e] + v.x * sb[e];
             }
-            uint8_t *qd = sm + kOffQ + qb * kTileBytes;
-#pragma unroll 2
-            for (int k = 0; k < 8; ++k) {
-                const int rr = rbase + 16 * k;
-                const uint32_t off = rr * 128 + ((ch ^ (rr & 7)) << 4);
-                const uint4 a4 = *reinterpret_cast<const uint4 *>(qt + off);
-                const uint4 b4 = *reinterpret_cast<const uint4 *>(qt + kHalfPlane + off);
-                const uint32_t *aw = reinterpret_cast<const uint32_t *>(&a4);
-                const uint32_t *bw = reinterpret_cast<const uint32_t *>(&b4);
-                uint4 lo, hi;
-                uint32_t *lw = reinterpret_cast<uint32_t *>(&lo);
-                uint32_t *hw = reinterpret_cast<uint32_t *>(&hi);
+            for (int tk = tok_first + tl; tk <= tok_first + (kRows + G - 1) / G; tk += 16) {
+                for (int gg = 0; gg < G; ++gg) {
+                    const int rr = tk * G + gg - R0;
+                    if (rr < 0 || rr >= kRows) continue;
+                    uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+                    if (tk <= tok_last) {
+                        const uint16_t *q =
+                            p.q_raw + (static_cast<size_t>(q0 + tk) * p.hq + kvh * G + gg) * kHeadDim;
+                        const uint4 a4 = *reinterpret_cast<const uint4 *>(q + 8 * ch);
+                        const uint4 b4 = *reinterpret_cast<const uint4 *>(q + kHalfDim + 8 * ch);
+                        const uint32_t *aw = reinterpret_cast<const uint32_t *>(&a4);
+                        const uint32_t *bw = reinterpret_cast<const uint32_t *>(&b4);
+                        uint32_t *lw = reinterpret_cast<uint32_t *>(&lo);
+                        uint32_t *hw = reinterpret_cast<uint32_t *>(&hi);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float a0 = bf16_lo(aw[e]), a1 = bf16_hi(aw[e]);
-                    const float b0 = bf16_lo(bw[e]), b1 = bf16_hi(bw[e]);
-                    const float c0 = cs[2 * e], s0 = sn[2 * e], c1 = cs[2 * e + 1], s1 = sn[2 * e + 1];
-                    lw[e] = pack_bf16(a0 * c0 - b0 * s0, a1 * c1 - b1 * s1);
-                    hw[e] = pack_bf16(b0 * c0 + a0 * s0, b1 * c1 + a1 * s1);
+                        for (int e = 0; e < 4; ++e) {
+                            const float a0 = bf16_lo(aw[e]) * p.scale_log2, a1 = bf16_hi(aw[e]) * p.scale_log2;
+                            const float b0 = bf16_lo(bw[e]) * p.scale_log2, b1 = bf16_hi(bw[e]) * p.scale_log2;
+                            const float c0 = cc[2 * e], s0 = ss[2 * e], c1 = cc[2 * e + 1], s1 = ss[2 * e + 1];
+                            lw[e] = pack_bf16(a0 * c0 - b0 * s0, a1 * c1 - b1 * s1);
+                            hw[e] = pack_bf16(b0 * c0 + a0 * s0, b1 * c1 + a1 * s1);
+                        }
+                    }
+                    const int tt = rr >> 7, rw = rr & 127;
+                    uint8_t *qd = sm + kOffQ + tt * kTileBytes;
+                    const uint32_t soff = rw * 128 + ((ch ^ (rw & 7)) << 4);
+                    *reinterpret_cast<uint4 *>(qd + soff) = lo;
+                    *reinterpret_cast<uint4 *>(qd + kHalfPlane + soff) = hi;
                 }
-                *reinterpret_cast<uint4 *>(qd + off) = lo;
-                *reinterpret_cast<uint4 *>(qd + kHalfPlane + off) = hi;
+                // advance the angle by 16 tokens
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float c2 = cc[e] * c16[e] - ss[e] * s16[e];
+                    ss[e] = ss[e] * c16[e] + cc[e] * s16[e];
+                    cc[e] = c2;
+                }
             }
             fence_proxy_async_smem();   // generic-proxy writes become visible to the tensor core
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_QFULL + qb]);
-            rot_sync();                 // segcs is rewritten for the next segment only after all reads
+            if (lane == 0) mbar_arrive(&bars[B_QFULL]);
+            rot_sync();                 // segcs may be rewritten only after every thread has read it
+            ++seg;
         }
     }
 
     // ================================================================ teardown
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 2) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tbase, 512);
     }
