@@ -28,10 +28,10 @@ namespace lazy {
 
 namespace {
 
-constexpr int kDecodeStages = 8;
 constexpr int kStageBytes = 2 * kBlockBytes;     // K + V of one word
 constexpr int kDecodeThreads = 160;               // 4 consumer warps + 1 producer warp
-constexpr size_t kDecodeSmem = kDecodeStages * kStageBytes + 1024;
+constexpr int kDefaultStages = 8;
+__host__ __device__ constexpr size_t decode_smem(int stages) { return size_t(stages) * kStageBytes + 1024; }
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -40,14 +40,20 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 // NT: groups of 8 query heads per KV head (1 for G <= 8, 2 for G <= 16, 4 for G <= 32).
 // PLAIN: keys come from a materialised copy indexed by table position, and the
 // query is rotated once at its absolute position (the comparison path).
-template <int NT, bool PLAIN>
+// Stage i of the ring holds word i mod kDecodeStages, and consumer warp kl takes
+// words i = kl (mod KW).  The ring size is a multiple of KW, so a stage always
+// returns to the same warp: a warp's parity wait on a stage can then never
+// run ahead of that stage's previous round (which another warp would own).
+template <int NT, bool PLAIN, int kDecodeStages>
 __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                       const __grid_constant__ CUtensorMap tmV,
                                                                       const AttnParams p) {
     constexpr int KW = 4 / NT;   // warps sharing the words of one head group
+    static_assert(kDecodeStages % 4 == 0, "the stage ring must be a multiple of the consumer warps");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *stages = align1024(smem_raw);
     __shared__ uint64_t full_bar[kDecodeStages], empty_bar[kDecodeStages];
+    __shared__ uint32_t stage_word[kDecodeStages], stage_meta[kDecodeStages];
     __shared__ double theta_s[kHalfDim];
 
     const int split = blockIdx.x, kvh = blockIdx.y, r = blockIdx.z;
@@ -96,11 +102,16 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
                 const uint32_t w = p.table[widx];
                 const uint32_t b = word_block(w);
                 issued = i + 1;
+                // the word and the block's metadata travel with the stage, so
+                // consumers read them from shared memory (the arrive releases them)
+                stage_word[st] = w;
                 if (b >= static_cast<uint32_t>(p.num_blocks)) {
+                    stage_meta[st] = 0u;
                     set_status(p.d_status, LAZY_DSTATUS_BAD_BLOCK);
                     mbar_arrive(&full_bar[st]);   // completes the phase with no data
                     continue;
                 }
+                stage_meta[st] = p.blk_meta[b];
                 mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
                 uint8_t *dst = stages + st * kStageBytes;
                 const int krow = PLAIN ? (widx * p.hkv + kvh) * kBlockTokens
@@ -151,10 +162,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
                 set_status(p.d_status, LAZY_DSTATUS_TIMEOUT);
                 break;
             }
-            const uint32_t w = p.table[wbase + lo + i];
+            const uint32_t w = stage_word[st];
             const uint32_t b = word_block(w);
             if (b < static_cast<uint32_t>(p.num_blocks)) {
-                const uint32_t meta = p.blk_meta[b];
+                const uint32_t meta = stage_meta[st];
                 const int off = word_offset(w);
                 const int off_rot = PLAIN ? 0 : off;
                 if (off_rot != cur_off) {
@@ -309,17 +320,35 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const AttnParams p)
     p.out[(static_cast<size_t>(r) * p.hq + h) * kHeadDim + d] = *reinterpret_cast<uint16_t *>(&ob);
 }
 
-template <int NT, bool PLAIN>
+template <int NT, bool PLAIN, int NS>
 cudaError_t launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, cudaStream_t s) {
-    auto kern = decode_split_kernel<NT, PLAIN>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmem);
+    auto kern = decode_split_kernel<NT, PLAIN, NS>;
+    const size_t smem = decode_smem(NS);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p.n_splits, p.hkv, p.num_req);
-    kern<<<grid, kDecodeThreads, kDecodeSmem, s>>>(tk, tv, p);
+    kern<<<grid, kDecodeThreads, smem, s>>>(tk, tv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     decode_combine_kernel<<<p.num_req * p.hq, kHeadDim, 0, s>>>(p);
     return cudaGetLastError();
+}
+
+// Pipeline depth (8 KiB stages per CTA, a multiple of 4); LAZY_ATTN_DECODE_STAGES
+// selects 4, 8 or 12 for tuning experiments.
+int decode_stages() {
+    const char *env = getenv("LAZY_ATTN_DECODE_STAGES");
+    const int v = env ? atoi(env) : kDefaultStages;
+    return (v == 4 || v == 12) ? v : kDefaultStages;
+}
+
+template <int NT, bool PLAIN>
+cudaError_t launch_decode_nt(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, cudaStream_t s) {
+    switch (decode_stages()) {
+    case 4: return launch_decode_t<NT, PLAIN, 4>(tk, tv, p, s);
+    case 12: return launch_decode_t<NT, PLAIN, 12>(tk, tv, p, s);
+    default: return launch_decode_t<NT, PLAIN, kDefaultStages>(tk, tv, p, s);
+    }
 }
 
 }  // namespace
@@ -345,13 +374,13 @@ cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const At
                           cudaStream_t s) {
     const int nt = p.group <= 8 ? 1 : (p.group <= 16 ? 2 : 4);
     if (plain) {
-        if (nt == 1) return launch_decode_t<1, true>(tk, tv, p, s);
-        if (nt == 2) return launch_decode_t<2, true>(tk, tv, p, s);
-        return launch_decode_t<4, true>(tk, tv, p, s);
+        if (nt == 1) return launch_decode_nt<1, true>(tk, tv, p, s);
+        if (nt == 2) return launch_decode_nt<2, true>(tk, tv, p, s);
+        return launch_decode_nt<4, true>(tk, tv, p, s);
     }
-    if (nt == 1) return launch_decode_t<1, false>(tk, tv, p, s);
-    if (nt == 2) return launch_decode_t<2, false>(tk, tv, p, s);
-    return launch_decode_t<4, false>(tk, tv, p, s);
+    if (nt == 1) return launch_decode_nt<1, false>(tk, tv, p, s);
+    if (nt == 2) return launch_decode_nt<2, false>(tk, tv, p, s);
+    return launch_decode_nt<4, false>(tk, tv, p, s);
 }
 
 }  // namespace lazy

@@ -10,21 +10,24 @@
 // again; this phase is compute-bound.
 //
 // Where the single relative rotation goes.  Keys sit in the pool rotated at
-// their local index j.  For every segment (document) that the table walk
-// enters, with logical offset o, the rotation warpgroup writes the query tile
-// Q'_i = R(p_i - o) q_i once; stored keys go from TMA to the tensor core
-// untouched and scores carry the angle (p_i - o - j) of eager RoPE attention.
-// The rewrite of the query tile overlaps the softmax of the segment's last
-// key tile, so it costs no tensor-core time.
+// their local index j.  Each CTA fixes a reference position P0 (its first
+// query token's position) and rotates its query tile once, Q'_i =
+// R(p_i - P0) q_i.  Every K tile, after TMA has landed it in shared memory,
+// gets one relative rotation R(o - P0) by its segment's offset o -- not a
+// reset to position 0 followed by a second rotation -- so that scores carry
+// the angle (p_i - o - j) of eager RoPE attention.  The rotation runs two
+// stages ahead of the MMAs that read the tile.  The plain (materialised)
+// path is the same kernel with that rotation removed: keys arrive rotated
+// at their absolute positions and the query is rotated at p_i.
 //
 // CTA = 256 query rows (two 128-row MMA tiles) of one KV head of one
 // request; rows are (token, head-in-group) pairs, token-major, so each K/V
 // tile loaded by TMA serves every query head of its group and both row
 // tiles.  16 warps:
 //   warp 0      K producer: walks the table once, publishes per-tile
-//               information (blocks, metadata, mask flags, segment flags) in
-//               a shared-memory ring, and TMA-loads K tiles (<= 8 blocks =
-//               128 keys of one segment) into 3 stages
+//               information (blocks, metadata, mask flag) in a shared-memory
+//               ring, and TMA-loads K tiles (<= 8 blocks = 128 keys of one
+//               segment) into 3 stages
 //   warp 1      V producer: TMA-loads V tiles into 2 stages
 //   warp 2      tensor-memory owner and MMA issuer, in the order
 //               QK0(j), PV1(j-1), QK1(j), PV0(j): while one softmax
@@ -34,7 +37,7 @@
 //               memory, mask, online softmax with lazy rescaling of O, P
 //               (bf16) written over the consumed S columns; epilogue O / l
 //   warps 8-11  softmax of row tile 1
-//   warps 12-15 query rotation, once per segment
+//   warps 12-15 rotations: the query tile once, then every K tile
 // Tensor memory (512 columns): S0 [0,128) (P0 = its first 64 columns),
 // S1 [128,256) (P1), O0 [256,384), O1 [384,512).
 #include <climits>
@@ -60,10 +63,10 @@ struct TileInfo {
     uint32_t meta[kTileBlocks];
     int n;       // blocks in the tile (1..8)
     int off;     // the segment's logical offset
-    int flags;   // kFull | kNewSeg | kSegEnd
+    int flags;   // kFull: every key of the tile is visible to every row of the CTA
     int pad;
 };
-constexpr int kFull = 1, kNewSeg = 2, kSegEnd = 4;
+constexpr int kFull = 1;
 
 constexpr int kOffQ = 0;                                     // 2 row tiles
 constexpr int kOffK = kOffQ + 2 * kTileBytes;                // 3 stages
@@ -71,20 +74,20 @@ constexpr int kOffV = kOffK + kKStages * kTileBytes;         // 2 stages
 constexpr int kOffInfo = kOffV + kVStages * kTileBytes;
 constexpr int kOffBar = kOffInfo + kInfoStages * static_cast<int>(sizeof(TileInfo));
 // barriers
-constexpr int B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_VFULL = B_KEMPTY + kKStages,
-              B_VEMPTY = B_VFULL + kVStages, B_IFULL = B_VEMPTY + kVStages, B_IEMPTY = B_IFULL + kInfoStages,
-              B_SFULL = B_IEMPTY + kInfoStages, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2, B_QFULL = B_ODONE + 2,
-              B_QEMPTY = B_QFULL + 1, B_DRAIN = B_QEMPTY + 1, kNumBars = B_DRAIN + 1;
+constexpr int B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_KROT = B_KEMPTY + kKStages,
+              B_VFULL = B_KROT + kKStages, B_VEMPTY = B_VFULL + kVStages, B_IFULL = B_VEMPTY + kVStages,
+              B_IEMPTY = B_IFULL + kInfoStages, B_SFULL = B_IEMPTY + kInfoStages, B_PFULL = B_SFULL + 2,
+              B_ODONE = B_PFULL + 2, B_QFULL = B_ODONE + 2, B_DRAIN = B_QFULL + 1, kNumBars = B_DRAIN + 1;
 constexpr int kOffTheta = kOffBar + kNumBars * 8;
-constexpr int kOffSeg = kOffTheta + kHalfDim * 8;
-constexpr int kOffMisc = kOffSeg + kHalfDim * 8;
+constexpr int kOffMisc = kOffTheta + kHalfDim * 8;
 constexpr int kSmemUse = kOffMisc + 16;
 constexpr size_t kTcSmem = kSmemUse + 1024;
 static_assert(kTcSmem <= 232448, "shared memory budget");
 static_assert(sizeof(TileInfo) == 80, "tile info layout");
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays below 2^8 between rescales
-// consumers of one tile-info entry: 8 softmax warps, the V producer, the MMA issuer
+// consumers of one tile-info entry: 8 softmax warps, the V producer, the MMA issuer, and on
+// the lazy path the 4 rotation warps
 constexpr int kInfoConsumers = 10;
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
@@ -107,7 +110,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     const bool ok = wait_or_abort(bar, parity, abort_flag, d_status);
     return __all_sync(0xffffffffu, ok);
 }
-__device__ __forceinline__ void rot_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 // Same decision for the 128 threads of the rotation warpgroup.
 __device__ __forceinline__ bool rot_all(bool ok) {
     uint32_t any_fail;
@@ -129,7 +131,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
     TileInfo *info = reinterpret_cast<TileInfo *>(sm + kOffInfo);
     double *theta_s = reinterpret_cast<double *>(sm + kOffTheta);
-    float2 *segcs = reinterpret_cast<float2 *>(sm + kOffSeg);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);
 
@@ -152,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         for (int i = 0; i < kKStages; ++i) {
             mbar_init(&bars[B_KFULL + i], 1);
             mbar_init(&bars[B_KEMPTY + i], 1);
+            mbar_init(&bars[B_KROT + i], 4);
         }
         for (int i = 0; i < kVStages; ++i) {
             mbar_init(&bars[B_VFULL + i], 1);
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         for (int i = 0; i < kInfoStages; ++i) {
             mbar_init(&bars[B_IFULL + i], 1);
-            mbar_init(&bars[B_IEMPTY + i], kInfoConsumers);
+            mbar_init(&bars[B_IEMPTY + i], kInfoConsumers + (PLAIN ? 0 : 4));
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bars[B_SFULL + t], 1);
@@ -167,7 +169,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             mbar_init(&bars[B_ODONE + t], 1);
         }
         mbar_init(&bars[B_QFULL], 4);
-        mbar_init(&bars[B_QEMPTY], 1);
         mbar_init(&bars[B_DRAIN], 1);
         *abort_flag = 0;
         if (mt == 0 && kvh == 0 && n_words > p.max_words) set_status(p.d_status, LAZY_DSTATUS_BAD_TABLE);
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         // ============================================================ table walk + K producer
         if (lane == 0) {
             tma_prefetch_desc(&tmK);
-            int issued = 0, prev_off = INT_MIN;
+            int issued = 0;
             for (int w = 0, j = 0; w < n_words; ++j) {
                 // the tile: up to 8 consecutive words that share one offset
                 uint32_t wd[kTileBlocks];
@@ -199,8 +200,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 for (int k = 1; k < kTileBlocks; ++k)
                     if (n == k && w + k < n_words && word_offset(wd[k]) == off) n = k + 1;
                 const int wn = w + n;
-                const int off_rot = PLAIN ? 0 : off;
-                const int next_rot = wn < n_words ? (PLAIN ? 0 : word_offset(tbl[wn])) : INT_MIN;
                 uint32_t mt_k[kTileBlocks];
                 bool full = n == kTileBlocks;
 #pragma unroll
@@ -212,9 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     full = full && meta_valid(mt_k[k]) == kBlockTokens &&
                            off + meta_j0(mt_k[k]) + kBlockTokens - 1 <= Pbase;
                 }
-                const int flags = (full ? kFull : 0) | (off_rot != prev_off ? kNewSeg : 0) |
-                                  (next_rot != off_rot ? kSegEnd : 0);
-                prev_off = off_rot;
+                const int flags = full ? kFull : 0;
                 // publish the tile information
                 const int is = j % kInfoStages;
                 if (!wait_or_abort(&bars[B_IEMPTY + is], ((j / kInfoStages) & 1) ^ 1, abort_flag, p.d_status)) break;
@@ -288,15 +285,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             const uint32_t idv = tc::idesc_bf16(128, 128, true);
             const uint32_t sQ = smem_u32(sm + kOffQ), sK = smem_u32(sm + kOffK), sV = smem_u32(sm + kOffV);
             const uint32_t tS[2] = {tbase, tbase + 128}, tO[2] = {tbase + 256, tbase + 384};
-            int seg = 0, prev_n = 0, j = 0;
+            // descriptors at offset 0 of each buffer; a byte offset b is added as b >> 4
+            // to the start-address field (no carry: shared addresses are below 2^18)
+            const uint64_t dQ0 = tc::smem_desc(sQ, 16, 1024), dK0 = tc::smem_desc(sK, 16, 1024);
+            const uint64_t dV0 = tc::smem_desc(sV, kHalfPlane, 1024);
+            int prev_n = 0, j = 0;
             bool ok = true;
             auto qk = [&](int t, int ks) {
-                const uint32_t qa = sQ + t * kTileBytes, kb = sK + ks * kTileBytes;
+                const uint64_t qa = dQ0 + static_cast<uint64_t>((t * kTileBytes) >> 4);
+                const uint64_t kb = dK0 + static_cast<uint64_t>((ks * kTileBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t o = (kk >> 2) * kHalfPlane + (kk & 3) * 32;
-                    tc::mma_ss(tS[t], tc::smem_desc(qa + o, 16, 1024), tc::smem_desc(kb + o, 16, 1024), idq,
-                               kk > 0 ? 1u : 0u);
+                    const uint64_t o = static_cast<uint64_t>(((kk >> 2) * kHalfPlane + (kk & 3) * 32) >> 4);
+                    tc::mma_ss(tS[t], qa + o, kb + o, idq, kk > 0 ? 1u : 0u);
                 }
                 tc::commit(&bars[B_SFULL + t]);
             };
@@ -306,31 +307,29 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 if (!wait_or_abort(&bars[B_VFULL + vs], (jj / kVStages) & 1, abort_flag, p.d_status)) return false;
                 if (!wait_or_abort(&bars[B_PFULL + t], jj & 1, abort_flag, p.d_status)) return false;
                 tc::fence_after_sync();
-                const uint32_t vb = sV + vs * kTileBytes;
+                const uint64_t vb = dV0 + static_cast<uint64_t>((vs * kTileBytes) >> 4);
                 for (int k = 0; k < n; ++k)
-                    tc::mma_ts(tO[t], tS[t] + 8 * k, tc::smem_desc(vb + k * kBoxBytes, kHalfPlane, 1024), idv,
+                    tc::mma_ts(tO[t], tS[t] + 8 * k, vb + static_cast<uint64_t>((k * kBoxBytes) >> 4), idv,
                                (jj > 0 || k > 0) ? 1u : 0u);
                 tc::commit(&bars[B_ODONE + t]);
                 if (t == 1) tc::commit(&bars[B_VEMPTY + vs]);   // V(jj) fully consumed
                 return true;
             };
+            ok = wait_or_abort(&bars[B_QFULL], 0, abort_flag, p.d_status);
             for (int w = 0; w < n_words && ok; ++j) {
                 const int is = j % kInfoStages;
                 if (!wait_or_abort(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) break;
-                const int n = info[is].n, flags = info[is].flags;
+                const int n = info[is].n;
                 mbar_arrive(&bars[B_IEMPTY + is]);
-                if (flags & kNewSeg) {
-                    if (!wait_or_abort(&bars[B_QFULL], seg & 1, abort_flag, p.d_status)) break;
-                    ++seg;
-                }
                 const int ks = j % kKStages;
-                if (!wait_or_abort(&bars[B_KFULL + ks], (j / kKStages) & 1, abort_flag, p.d_status)) break;
+                // the plain path uses keys as loaded; the lazy path waits for their rotation
+                uint64_t *kready = PLAIN ? &bars[B_KFULL + ks] : &bars[B_KROT + ks];
+                if (!wait_or_abort(kready, (j / kKStages) & 1, abort_flag, p.d_status)) break;
                 tc::fence_after_sync();
                 qk(0, ks);
                 if (j >= 1 && !(ok = pv(1, j - 1, prev_n))) break;
                 qk(1, ks);
                 tc::commit(&bars[B_KEMPTY + ks]);
-                if (flags & kSegEnd) tc::commit(&bars[B_QEMPTY]);
                 if (!(ok = pv(0, j, n))) break;
                 prev_n = n;
                 w += n;
@@ -370,22 +369,30 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             if (lane == 0) mbar_arrive(&bars[B_IEMPTY + is]);
             if (!warp_wait(&bars[B_SFULL + t], j & 1, abort_flag, p.d_status)) { ok = false; break; }
             tc::fence_after_sync();
-            // pass 1: masked row maximum (S_t(j) complete implies PV_t(j-1) complete)
+            // pass 1: masked row maximum (S_t(j) complete implies PV_t(j-1) complete).
+            // Two 32-column loads are in flight per wait.
             float tmax = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t x[32];
-                tc::ld32(tS + lane_off + 32 * c, x);
+            for (int c = 0; c < 4; c += 2) {
+                uint32_t xa[32], xb[32];
+                tc::ld32(tS + lane_off + 32 * c, xa);
+                tc::ld32(tS + lane_off + 32 * (c + 1), xb);
                 tc::wait_ld();
                 if (full) {
+                    float m0 = __uint_as_float(xa[0]), m1 = __uint_as_float(xb[0]);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, __uint_as_float(x[e]));
+                    for (int e = 1; e < 32; ++e) {
+                        m0 = fmaxf(m0, __uint_as_float(xa[e]));
+                        m1 = fmaxf(m1, __uint_as_float(xb[e]));
+                    }
+                    tmax = fmaxf(tmax, fmaxf(m0, m1));
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
+                    for (int e = 0; e < 64; ++e) {
                         const int col = 32 * c + e, k = col >> 4, si = col & 15;
+                        const uint32_t xv = e < 32 ? xa[e] : xb[e - 32];
                         const bool vis = si < knv[k] && off + kj0[k] + si <= prow;
-                        tmax = vis ? fmaxf(tmax, __uint_as_float(x[e])) : tmax;
+                        tmax = vis ? fmaxf(tmax, __uint_as_float(xv)) : tmax;
                     }
                 }
             }
@@ -412,23 +419,44 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             // pass 2: P = 2^(S - m) as bf16 pairs over the consumed S columns, row sum in fp32
             float lsum = 0.f;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t x[32], pk[16];
-                tc::ld32(tS + lane_off + 32 * c, x);
+            for (int c = 0; c < 4; c += 2) {
+                uint32_t xa[32], xb[32];
+                tc::ld32(tS + lane_off + 32 * c, xa);
+                tc::ld32(tS + lane_off + 32 * (c + 1), xb);
                 tc::wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float pr[2];
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t *x = h == 0 ? xa : xb;
+                    const int cc = c + h;
+                    uint32_t pk[16];
+                    if (full) {
+                        float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int col = 32 * c + 2 * e + h, k = col >> 4, si = col & 15;
-                        const bool vis = full || (si < knv[k] && off + kj0[k] + si <= prow);
-                        pr[h] = vis ? fast_exp2(__uint_as_float(x[2 * e + h]) - mu) : 0.f;
+                        for (int e = 0; e < 16; ++e) {
+                            const float p0 = fast_exp2(__uint_as_float(x[2 * e]) - mu);
+                            const float p1 = fast_exp2(__uint_as_float(x[2 * e + 1]) - mu);
+                            ls0 += p0;
+                            ls1 += p1;
+                            pk[e] = pack_bf16(p0, p1);
+                        }
+                        lsum += ls0 + ls1;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            float pr[2];
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const int col = 32 * cc + 2 * e + hh, k = col >> 4, si = col & 15;
+                                const bool vis = si < knv[k] && off + kj0[k] + si <= prow;
+                                pr[hh] = vis ? fast_exp2(__uint_as_float(x[2 * e + hh]) - mu) : 0.f;
+                            }
+                            lsum += pr[0] + pr[1];
+                            pk[e] = pack_bf16(pr[0], pr[1]);
+                        }
                     }
-                    lsum += pr[0] + pr[1];
-                    pk[e] = pack_bf16(pr[0], pr[1]);
+                    // P columns 16cc..16cc+15 were S columns already read in this or an earlier chunk
+                    tc::st16(tS + lane_off + 16 * cc, pk);
                 }
-                tc::st16(tS + lane_off + 16 * c, pk);   // columns already read in this or an earlier chunk
             }
             l_run += lsum;
             tc::wait_st();
@@ -469,52 +497,69 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             }
         }
     } else if (warp >= 12) {
-        // ============================================================ query rotation
+        // ============================================================ rotations
+        // (1) Q'_i = R(p_i - P0) q_i once per CTA (R(p_i) on the plain path), P0 =
+        //     the CTA's first query position.  Thread (ch, rb) writes pairs
+        //     8ch..8ch+7 of rows rb + 16k of each row tile; between rows rb + 16k
+        //     and rb + 16(k+1) the token advances by dlo = 16 / G or dlo + 1
+        //     tokens, so angles advance by rotation with two step tables.
+        // (2) lazy path only: every K tile, once TMA has landed it, is rotated
+        //     in shared memory by (o - P0) -- one relative rotation per tile --
+        //     so that scores carry the angle (p_i - o - j).
         const int tid = threadIdx.x - 384;
-        const int ch = tid & 7;         // pairs 8ch .. 8ch+7
-        const int tl = tid >> 3;        // tokens tok_first + tl + 16k
-        // per-thread constants: rotation by 16 tokens, and by (tl tokens) from the CTA's first token
-        float c16[8], s16[8], cb[8], sb[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            rope_cos_sin(16, theta_s[8 * ch + e], c16[e], s16[e]);
-            rope_cos_sin(tl, theta_s[8 * ch + e], cb[e], sb[e]);
-        }
-        int seg = 0, cur = INT_MIN;
-        for (int w = 0; w < n_words; ++w) {
-            const int off_rot = PLAIN ? 0 : word_offset(tbl[w]);
-            if (off_rot == cur) continue;
-            cur = off_rot;
-            bool okw = true;
-            if (seg >= 1) okw = wait_or_abort(&bars[B_QEMPTY], (seg - 1) & 1, abort_flag, p.d_status);
-            if (!rot_all(okw)) break;
-            // the segment's rotation R(P - o), one pair per thread
-            if (tid < kHalfDim) {
-                float c, s;
-                rope_cos_sin(Pbase - off_rot, theta_s[tid], c, s);
-                segcs[tid] = make_float2(c, s);
-            }
-            rot_sync();
-            // angle of this thread's first token: R(P - o) composed with R(tl)
-            float cc[8], ss[8];
+        const int ch = tid & 7;
+        const int rb = tid >> 3;
+        {
+            const int dlo = 16 / G;
+            float cA[8], sA[8], cB[8], sB[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float2 v = segcs[8 * ch + e];
-                cc[e] = v.x * cb[e] - v.y * sb[e];
-                ss[e] = v.y * cb[e] + v.x * sb[e];
+                rope_cos_sin(dlo, theta_s[8 * ch + e], cA[e], sA[e]);
+                rope_cos_sin(dlo + 1, theta_s[8 * ch + e], cB[e], sB[e]);
             }
-            for (int tk = tok_first + tl; tk <= tok_first + (kRows + G - 1) / G; tk += 16) {
-                for (int gg = 0; gg < G; ++gg) {
-                    const int rr = tk * G + gg - R0;
-                    if (rr < 0 || rr >= kRows) continue;
-                    uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
-                    if (tk <= tok_last) {
-                        const uint16_t *q =
-                            p.q_raw + (static_cast<size_t>(q0 + tk) * p.hq + kvh * G + gg) * kHeadDim;
-                        const uint4 a4 = *reinterpret_cast<const uint4 *>(q + 8 * ch);
-                        const uint4 b4 = *reinterpret_cast<const uint4 *>(q + kHalfDim + 8 * ch);
-                        const uint32_t *aw = reinterpret_cast<const uint32_t *>(&a4);
-                        const uint32_t *bw = reinterpret_cast<const uint32_t *>(&b4);
+            const int qref = PLAIN ? 0 : Pbase;
+            for (int t = 0; t < 2; ++t) {
+                const int rowbase = R0 + kTileRows * t + rb;   // global row of k = 0
+                int tk_prev = rowbase / G;
+                float cc[8], ss[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) rope_cos_sin(pos0 + tk_prev - qref, theta_s[8 * ch + e], cc[e], ss[e]);
+                uint8_t *qd = sm + kOffQ + t * kTileBytes;
+#pragma unroll 1
+                for (int kg = 0; kg < 8; kg += 4) {
+                    // issue the global loads of four rows before using any of them
+                    uint4 a4[4], b4[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int R = rowbase + 16 * (kg + u);
+                        a4[u] = make_uint4(0, 0, 0, 0);
+                        b4[u] = make_uint4(0, 0, 0, 0);
+                        if (R < T * G) {
+                            const uint16_t *q = p.q_raw +
+                                                (static_cast<size_t>(q0 + R / G) * p.hq + kvh * G + R % G) * kHeadDim;
+                            a4[u] = *reinterpret_cast<const uint4 *>(q + 8 * ch);
+                            b4[u] = *reinterpret_cast<const uint4 *>(q + kHalfDim + 8 * ch);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int k = kg + u;
+                        const int R = rowbase + 16 * k;
+                        const int tk = R / G;
+                        if (k > 0 && tk != tk_prev) {
+                            const bool big = tk - tk_prev != dlo;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const float sc = big ? cB[e] : cA[e], sn = big ? sB[e] : sA[e];
+                                const float c2 = cc[e] * sc - ss[e] * sn;
+                                ss[e] = ss[e] * sc + cc[e] * sn;
+                                cc[e] = c2;
+                            }
+                            tk_prev = tk;
+                        }
+                        const uint32_t *aw = reinterpret_cast<const uint32_t *>(&a4[u]);
+                        const uint32_t *bw = reinterpret_cast<const uint32_t *>(&b4[u]);
+                        uint4 lo, hi;
                         uint32_t *lw = reinterpret_cast<uint32_t *>(&lo);
                         uint32_t *hw = reinterpret_cast<uint32_t *>(&hi);
 #pragma unroll
@@ -525,26 +570,65 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                             lw[e] = pack_bf16(a0 * c0 - b0 * s0, a1 * c1 - b1 * s1);
                             hw[e] = pack_bf16(b0 * c0 + a0 * s0, b1 * c1 + a1 * s1);
                         }
+                        const int rw = rb + 16 * k;
+                        const uint32_t soff = rw * 128 + ((ch ^ (rw & 7)) << 4);
+                        *reinterpret_cast<uint4 *>(qd + soff) = lo;
+                        *reinterpret_cast<uint4 *>(qd + kHalfPlane + soff) = hi;
                     }
-                    const int tt = rr >> 7, rw = rr & 127;
-                    uint8_t *qd = sm + kOffQ + tt * kTileBytes;
-                    const uint32_t soff = rw * 128 + ((ch ^ (rw & 7)) << 4);
-                    *reinterpret_cast<uint4 *>(qd + soff) = lo;
-                    *reinterpret_cast<uint4 *>(qd + kHalfPlane + soff) = hi;
-                }
-                // advance the angle by 16 tokens
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float c2 = cc[e] * c16[e] - ss[e] * s16[e];
-                    ss[e] = ss[e] * c16[e] + cc[e] * s16[e];
-                    cc[e] = c2;
                 }
             }
             fence_proxy_async_smem();   // generic-proxy writes become visible to the tensor core
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_QFULL]);
-            rot_sync();                 // segcs may be rewritten only after every thread has read it
-            ++seg;
+        }
+        if (!PLAIN) {
+            int cur = INT_MIN;
+            float kc[8], kn[8];
+            for (int w = 0, j = 0; w < n_words; ++j) {
+                const int is = j % kInfoStages;
+                bool okw = wait_or_abort(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status);
+                if (!rot_all(okw)) break;
+                const int n = info[is].n, off = info[is].off;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_IEMPTY + is]);
+                if (off != cur) {
+                    cur = off;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) rope_cos_sin(off - Pbase, theta_s[8 * ch + e], kc[e], kn[e]);
+                }
+                const int ks = j % kKStages;
+                okw = wait_or_abort(&bars[B_KFULL + ks], (j / kKStages) & 1, abort_flag, p.d_status);
+                if (!rot_all(okw)) break;
+                uint8_t *kt = sm + kOffK + ks * kTileBytes;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int row = rb + 16 * k;   // key row of the tile
+                    if (row < kBlockTokens * n) {
+                        const uint32_t soff = row * 128 + ((ch ^ (row & 7)) << 4);
+                        const uint4 a4 = *reinterpret_cast<const uint4 *>(kt + soff);
+                        const uint4 b4 = *reinterpret_cast<const uint4 *>(kt + kHalfPlane + soff);
+                        const uint32_t *aw = reinterpret_cast<const uint32_t *>(&a4);
+                        const uint32_t *bw = reinterpret_cast<const uint32_t *>(&b4);
+                        uint4 lo, hi;
+                        uint32_t *lw = reinterpret_cast<uint32_t *>(&lo);
+                        uint32_t *hw = reinterpret_cast<uint32_t *>(&hi);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float a0 = bf16_lo(aw[e]), a1 = bf16_hi(aw[e]);
+                            const float b0 = bf16_lo(bw[e]), b1 = bf16_hi(bw[e]);
+                            const float c0 = kc[2 * e], s0 = kn[2 * e], c1 = kc[2 * e + 1], s1 = kn[2 * e + 1];
+                            lw[e] = pack_bf16(a0 * c0 - b0 * s0, a1 * c1 - b1 * s1);
+                            hw[e] = pack_bf16(b0 * c0 + a0 * s0, b1 * c1 + a1 * s1);
+                        }
+                        *reinterpret_cast<uint4 *>(kt + soff) = lo;
+                        *reinterpret_cast<uint4 *>(kt + kHalfPlane + soff) = hi;
+                    }
+                }
+                fence_proxy_async_smem();   // the tensor core reads the rotated tile
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_KROT + ks]);
+                w += n;
+            }
         }
     }
 
