@@ -29,10 +29,9 @@
 //               ring, and TMA-loads K tiles (<= 8 blocks = 128 keys of one
 //               segment) into 3 stages
 //   warp 1      V producer: TMA-loads V tiles into 2 stages
-//   warp 2      tensor-memory owner and MMA issuer, in the order
-//               QK0(j), PV1(j-1), QK1(j), PV0(j): while one softmax
-//               warpgroup works on its tile the tensor core runs the other's
-//   warp 3      idle
+//   warps 2, 3  MMA issuers for row tiles 0 and 1 (warp 2 also owns tensor
+//               memory): QK_t(j) then PV_t(j); while one softmax warpgroup
+//               works on its tile the tensor core runs the other tile's MMAs
 //   warps 4-7   softmax of row tile 0, one thread per row: S from tensor
 //               memory, mask, online softmax with lazy rescaling of O, P
 //               (bf16) written over the consumed S columns; epilogue O / l
@@ -86,9 +85,9 @@ static_assert(kTcSmem <= 232448, "shared memory budget");
 static_assert(sizeof(TileInfo) == 80, "tile info layout");
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays below 2^8 between rescales
-// consumers of one tile-info entry: 8 softmax warps, the V producer, the MMA issuer, and on
-// the lazy path the 4 rotation warps
-constexpr int kInfoConsumers = 10;
+// consumers of one tile-info entry: 8 softmax warps, the V producer, the two MMA warps, and
+// on the lazy path the 4 rotation warps
+constexpr int kInfoConsumers = 11;
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -152,12 +151,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     if (threadIdx.x == 0) {
         for (int i = 0; i < kKStages; ++i) {
             mbar_init(&bars[B_KFULL + i], 1);
-            mbar_init(&bars[B_KEMPTY + i], 1);
+            mbar_init(&bars[B_KEMPTY + i], 2);   // one commit per MMA warp
             mbar_init(&bars[B_KROT + i], 4);
         }
         for (int i = 0; i < kVStages; ++i) {
             mbar_init(&bars[B_VFULL + i], 1);
-            mbar_init(&bars[B_VEMPTY + i], 1);
+            mbar_init(&bars[B_VEMPTY + i], 2);   // one commit per MMA warp
         }
         for (int i = 0; i < kInfoStages; ++i) {
             mbar_init(&bars[B_IFULL + i], 1);
@@ -169,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             mbar_init(&bars[B_ODONE + t], 1);
         }
         mbar_init(&bars[B_QFULL], 4);
-        mbar_init(&bars[B_DRAIN], 1);
+        mbar_init(&bars[B_DRAIN], 2);
         *abort_flag = 0;
         if (mt == 0 && kvh == 0 && n_words > p.max_words) set_status(p.d_status, LAZY_DSTATUS_BAD_TABLE);
         fence_barrier_init();
@@ -278,45 +277,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             for (int j = max(0, issued - kVStages); j < issued; ++j)
                 mbar_wait(&bars[B_VFULL + j % kVStages], (j / kVStages) & 1);
         }
-    } else if (warp == 2) {
-        // ============================================================ MMA issuer
+    } else if (warp == 2 || warp == 3) {
+        // ============================================================ MMA issuers
+        // Warp 2 issues row tile 0's MMAs, warp 3 row tile 1's: two independent
+        // issuers keep more MMAs in flight than one (measured on B200: about 86
+        // instead of about 100 cycles per 128x128x16 MMA).  Per tile the order
+        // is QK_t(j), then PV_t(j) once softmax t has written P_t(j); QK_t(j+1)
+        // follows PV_t(j) in issue order, which is what lets P_t live in S_t.
         if (lane == 0) {
+            const int t = warp - 2;
             const uint32_t idq = tc::idesc_bf16(128, 128, false);
             const uint32_t idv = tc::idesc_bf16(128, 128, true);
             const uint32_t sQ = smem_u32(sm + kOffQ), sK = smem_u32(sm + kOffK), sV = smem_u32(sm + kOffV);
-            const uint32_t tS[2] = {tbase, tbase + 128}, tO[2] = {tbase + 256, tbase + 384};
+            const uint32_t tS = tbase + 128 * t, tO = tbase + 256 + 128 * t;
             // descriptors at offset 0 of each buffer; a byte offset b is added as b >> 4
             // to the start-address field (no carry: shared addresses are below 2^18)
-            const uint64_t dQ0 = tc::smem_desc(sQ, 16, 1024), dK0 = tc::smem_desc(sK, 16, 1024);
+            const uint64_t dQ = tc::smem_desc(sQ + t * kTileBytes, 16, 1024), dK0 = tc::smem_desc(sK, 16, 1024);
             const uint64_t dV0 = tc::smem_desc(sV, kHalfPlane, 1024);
-            int prev_n = 0, j = 0;
-            bool ok = true;
-            auto qk = [&](int t, int ks) {
-                const uint64_t qa = dQ0 + static_cast<uint64_t>((t * kTileBytes) >> 4);
-                const uint64_t kb = dK0 + static_cast<uint64_t>((ks * kTileBytes) >> 4);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t o = static_cast<uint64_t>(((kk >> 2) * kHalfPlane + (kk & 3) * 32) >> 4);
-                    tc::mma_ss(tS[t], qa + o, kb + o, idq, kk > 0 ? 1u : 0u);
-                }
-                tc::commit(&bars[B_SFULL + t]);
-            };
-            // O_t += P_t V(jj); P_t occupies the first 64 columns of S_t
-            auto pv = [&](int t, int jj, int n) -> bool {
-                const int vs = jj % kVStages;
-                if (!wait_or_abort(&bars[B_VFULL + vs], (jj / kVStages) & 1, abort_flag, p.d_status)) return false;
-                if (!wait_or_abort(&bars[B_PFULL + t], jj & 1, abort_flag, p.d_status)) return false;
-                tc::fence_after_sync();
-                const uint64_t vb = dV0 + static_cast<uint64_t>((vs * kTileBytes) >> 4);
-                for (int k = 0; k < n; ++k)
-                    tc::mma_ts(tO[t], tS[t] + 8 * k, vb + static_cast<uint64_t>((k * kBoxBytes) >> 4), idv,
-                               (jj > 0 || k > 0) ? 1u : 0u);
-                tc::commit(&bars[B_ODONE + t]);
-                if (t == 1) tc::commit(&bars[B_VEMPTY + vs]);   // V(jj) fully consumed
-                return true;
-            };
-            ok = wait_or_abort(&bars[B_QFULL], 0, abort_flag, p.d_status);
-            for (int w = 0; w < n_words && ok; ++j) {
+            bool ok = wait_or_abort(&bars[B_QFULL], 0, abort_flag, p.d_status);
+            for (int w = 0, j = 0; w < n_words && ok; ++j) {
                 const int is = j % kInfoStages;
                 if (!wait_or_abort(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) break;
                 const int n = info[is].n;
@@ -326,15 +305,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 uint64_t *kready = PLAIN ? &bars[B_KFULL + ks] : &bars[B_KROT + ks];
                 if (!wait_or_abort(kready, (j / kKStages) & 1, abort_flag, p.d_status)) break;
                 tc::fence_after_sync();
-                qk(0, ks);
-                if (j >= 1 && !(ok = pv(1, j - 1, prev_n))) break;
-                qk(1, ks);
+                const uint64_t kb = dK0 + static_cast<uint64_t>((ks * kTileBytes) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t o = static_cast<uint64_t>(((kk >> 2) * kHalfPlane + (kk & 3) * 32) >> 4);
+                    tc::mma_ss(tS, dQ + o, kb + o, idq, kk > 0 ? 1u : 0u);
+                }
+                tc::commit(&bars[B_SFULL + t]);
                 tc::commit(&bars[B_KEMPTY + ks]);
-                if (!(ok = pv(0, j, n))) break;
-                prev_n = n;
+                // O_t += P_t V(j); P_t occupies the first 64 columns of S_t
+                const int vs = j % kVStages;
+                if (!wait_or_abort(&bars[B_VFULL + vs], (j / kVStages) & 1, abort_flag, p.d_status)) break;
+                if (!wait_or_abort(&bars[B_PFULL + t], j & 1, abort_flag, p.d_status)) break;
+                tc::fence_after_sync();
+                const uint64_t vb = dV0 + static_cast<uint64_t>((vs * kTileBytes) >> 4);
+                for (int k = 0; k < n; ++k)
+                    tc::mma_ts(tO, tS + 8 * k, vb + static_cast<uint64_t>((k * kBoxBytes) >> 4), idv,
+                               (j > 0 || k > 0) ? 1u : 0u);
+                tc::commit(&bars[B_ODONE + t]);
+                tc::commit(&bars[B_VEMPTY + vs]);
                 w += n;
             }
-            if (ok && j >= 1 && !*abort_flag) pv(1, j - 1, prev_n);
             // every MMA this thread issued has completed before tensor memory is freed
             tc::commit(&bars[B_DRAIN]);
             mbar_wait(&bars[B_DRAIN], 0);
