@@ -327,6 +327,10 @@ def run_ours(args):
         result["prefill"] = run_prefill(args, world, peaks, peak_src, flush)
         result["gpu_launches"] += 2 * args.steps
 
+    # ---------------------------------------------------------------- other workloads (optional)
+    if args.extended:
+        result["extended"] = run_extended(args, world, peaks, peak_src, flush)
+
     # ---------------------------------------------------------------- CPU baseline (oracle), rank 0, N = 1
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline(wl, step, args.cpu_requests)
@@ -445,6 +449,57 @@ def run_prefill(args, world, peaks, peak_src, flush):
     }
 
 
+def run_extended(args, world, peaks, peak_src, flush):
+    """Decode 70B shapes (Zipf 1.2 and uniform popularity) and the mixed 8B serving
+    step (32 prefill chunks + 192 decodes, 1 GiB pool; GQA and MQA): per step
+    kind, the attention time and its throughput against the roofline."""
+    import torch
+
+    from position_agnostic_paged_b200 import accounting
+    from position_agnostic_paged_b200 import workloads as W
+    from position_agnostic_paged_b200.runner import DevicePool, DeviceStep
+
+    out = {}
+    for name in ("decode_70b", "decode_70b_uniform", "mixed_8b", "mixed_8b_mqa"):
+        t0 = time.time()
+        wl = W.make(name)
+        pool = DevicePool(wl).setup()
+        entry = {"unique_docs": wl.info["unique_docs_used"], "pool_blocks": wl.num_blocks}
+        for step in wl.steps:
+            ds = DeviceStep(pool, step)
+            _prepare_step_writes(ds)
+
+            def st(ev):
+                ds.write_new_tokens_dev()
+                if ev is not None:
+                    ev[0].record()
+                ds.attend()
+                if ev is not None:
+                    ev[1].record()
+
+            total, inner = timed_steps(st, args.steps, args.warmup, flush, world, inner=True)
+            attn = max_over_ranks(world, float(np.mean(inner)))
+            if step.kind == "decode":
+                b = accounting.decode_kv_bytes(step.kv_len, wl.hkv, wl.d)
+                entry["decode"] = {"requests": step.num_req, "kv_bytes": b, "attn_ms": round(attn, 5),
+                                   "GB/s": round(b / (attn * 1e-3) / 1e9, 1),
+                                   "frac_of_hbm_peak": round(b / (attn * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+            else:
+                f = accounting.prefill_flops(step.visible_pairs, wl.hq, wl.d)
+                tf = f / (attn * 1e-3) / 1e12
+                entry["prefill"] = {"requests": step.num_req, "flops": f, "attn_ms": round(attn, 5),
+                                    "TFLOP/s": round(tf, 1),
+                                    "frac_of_bf16_peak": round(tf / peaks.get("bf16_tflops", 1590.0), 4)}
+            del ds
+        if pool.status() != 0:
+            raise SystemExit(f"device status {pool.status()} in {name}")
+        del pool
+        torch.cuda.empty_cache()
+        log(f"[extended] {name} done in {time.time() - t0:.1f}s")
+        out[name] = entry
+    return out
+
+
 def cpu_baseline(wl, step, n_req: int):
     import oracle
     from position_agnostic_paged_b200 import accounting
@@ -520,6 +575,8 @@ def main():
     ap.add_argument("--no-compare", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--extended", action="store_true",
+                    help="also time decode 70B (Zipf 1.2 and uniform) and the mixed 8B step (GQA, MQA)")
     ap.add_argument("--cpu-requests", type=int, default=64)
     ap.add_argument("--ref-requests", type=int, default=2)
     args = ap.parse_args()
