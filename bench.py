@@ -445,7 +445,7 @@ def run_prefill(args, world, peaks, peak_src, flush):
         "algorithmic_flops_per_launch": flops,
         "roofline": {"bound": "tensor", "kernel": "lazy_prefill_attn", "achieved": round(achieved, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_source": peak_src,
-                     "traffic": traffic_for("prefill_8b", "prefill_mma.cu")},
+                     "traffic": traffic_for("prefill_8b", "prefill_tc.cu")},
     }
 
 

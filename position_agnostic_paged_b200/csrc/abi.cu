@@ -51,6 +51,21 @@ bool make_rows_map(CUtensorMap *map, const void *base, int64_t rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same pool viewed as (d, token, head, block): one box covers 8 consecutive
+// blocks of one head and one 64-element half (16 KiB), laid out in shared memory
+// exactly like 8 single-block boxes stacked.
+bool make_blocks_map(CUtensorMap *map, const void *base, int64_t nblocks, int hkv) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || nblocks <= 0 || hkv <= 0) return false;
+    cuuint64_t dims[4] = {128, 16, static_cast<cuuint64_t>(hkv), static_cast<cuuint64_t>(nblocks)};
+    cuuint64_t strides[3] = {256, 4096, static_cast<cuuint64_t>(hkv) * 4096};
+    cuuint32_t box[4] = {64, 16, 1, 8};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int check_cfg(const lazy_attn_cfg *cfg) {
     if (!cfg) return LAZY_EINVAL;
     if (cfg->head_dim != 128 || cfg->block_size != 16) return LAZY_ESHAPE;
@@ -166,13 +181,16 @@ int prefill_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t 
     p.max_q = max_q;
     p.k_rows = static_cast<int>(k_rows);
     p.v_rows = static_cast<int>(static_cast<int64_t>(num_blocks) * p.hkv * 16);
-    CUtensorMap tk, tv;
+    CUtensorMap tk, tv, tk8, tv8;
     if (!make_rows_map(&tk, k_src, k_rows) || !make_rows_map(&tv, v_pool, p.v_rows)) return LAZY_ECUDA;
+    if (!make_blocks_map(&tk8, k_src, k_rows / (16 * p.hkv), p.hkv) ||
+        !make_blocks_map(&tv8, v_pool, num_blocks, p.hkv))
+        return LAZY_ECUDA;
     // each request writes exactly its own query tokens' rows
     const char *impl = getenv("LAZY_ATTN_PREFILL_IMPL");
     if (impl && impl[0] == 'm')
         return launch_rc(launch_prefill(tk, tv, p, plain, static_cast<cudaStream_t>(stream)));
-    return launch_rc(launch_prefill_tc(tk, tv, p, plain, static_cast<cudaStream_t>(stream)));
+    return launch_rc(launch_prefill_tc(tk, tv, tk8, tv8, p, plain, static_cast<cudaStream_t>(stream)));
 }
 
 }  // namespace

@@ -23,20 +23,24 @@
 // CTA = 256 query rows (two 128-row MMA tiles) of one KV head of one
 // request; rows are (token, head-in-group) pairs, token-major, so each K/V
 // tile loaded by TMA serves every query head of its group and both row
-// tiles.  16 warps:
+// tiles.  16 warps in four warpgroups, registers rebalanced with setmaxnreg
+// (producers/MMA 72, softmax 192, K rotation 56 per thread):
 //   warp 0      K producer: walks the table once, publishes per-tile
 //               information (blocks, metadata, mask flag) in a shared-memory
 //               ring, and TMA-loads K tiles (<= 8 blocks = 128 keys of one
-//               segment) into 3 stages
-//   warp 1      V producer: TMA-loads V tiles into 2 stages
+//               segment) into 3 stages -- two 16 KiB boxes when the tile's
+//               blocks are consecutive in the pool, else two 2 KiB boxes per
+//               block
+//   warp 1      V producer: the same for V tiles, 2 stages
 //   warps 2, 3  MMA issuers for row tiles 0 and 1 (warp 2 also owns tensor
-//               memory): QK_t(j) then PV_t(j); while one softmax warpgroup
-//               works on its tile the tensor core runs the other tile's MMAs
-//   warps 4-7   softmax of row tile 0, one thread per row: S from tensor
-//               memory, mask, online softmax with lazy rescaling of O, P
-//               (bf16) written over the consumed S columns; epilogue O / l
-//   warps 8-11  softmax of row tile 1
-//   warps 12-15 rotations: the query tile once, then every K tile
+//               memory): QK_t(j) then PV_t(j)
+//   warps 4-7   row tile 0, one thread per row: first the rotated query rows
+//               of the tile, then per K tile the online softmax with the whole
+//               128-column score row in registers (one tensor-memory load,
+//               mask, max, 2^(S - m), one store of P over the consumed S
+//               columns), lazy rescaling of O; epilogue O / l
+//   warps 8-11  the same for row tile 1
+//   warps 12-15 K rotation: every K tile once, in shared memory
 // Tensor memory (512 columns): S0 [0,128) (P0 = its first 64 columns),
 // S1 [128,256) (P1), O0 [256,384), O1 [384,512).
 #include <climits>
@@ -104,11 +108,28 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
     set_status(d_status, LAZY_DSTATUS_TIMEOUT);
     return false;
 }
+// 4D tiled load: 8 consecutive blocks of one head, one 64-element half (16 KiB).
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int x, int y, int h, int b,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(h), "r"(b), "r"(smem_u32(bar))
+        : "memory");
+}
 // Same decision for every lane of the warp.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *d_status) {
     const bool ok = wait_or_abort(bar, parity, abort_flag, d_status);
     return __all_sync(0xffffffffu, ok);
 }
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N)); }
+// Register split (launch: 512 threads x 128 registers): producers + MMA warpgroup, two
+// softmax warpgroups, rotation warpgroup.
+constexpr int kProducerRegs = 72, kSoftmaxRegs = 192, kRotRegs = 56;
+static_assert(kProducerRegs * 128 + 2 * kSoftmaxRegs * 128 + kRotRegs * 128 <= 65536, "register split");
 // Same decision for the 128 threads of the rotation warpgroup.
 __device__ __forceinline__ bool rot_all(bool ok) {
     uint32_t any_fail;
@@ -124,6 +145,8 @@ __device__ __forceinline__ bool rot_all(bool ok) {
 template <bool PLAIN>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                  const __grid_constant__ CUtensorMap tmV,
+                                                                 const __grid_constant__ CUtensorMap tmK8,
+                                                                 const __grid_constant__ CUtensorMap tmV8,
                                                                  const AttnParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
@@ -151,12 +174,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     if (threadIdx.x == 0) {
         for (int i = 0; i < kKStages; ++i) {
             mbar_init(&bars[B_KFULL + i], 1);
-            mbar_init(&bars[B_KEMPTY + i], 2);   // one commit per MMA warp
+            mbar_init(&bars[B_KEMPTY + i], 2);
             mbar_init(&bars[B_KROT + i], 4);
         }
         for (int i = 0; i < kVStages; ++i) {
             mbar_init(&bars[B_VFULL + i], 1);
-            mbar_init(&bars[B_VEMPTY + i], 2);   // one commit per MMA warp
+            mbar_init(&bars[B_VEMPTY + i], 2);
         }
         for (int i = 0; i < kInfoStages; ++i) {
             mbar_init(&bars[B_IFULL + i], 1);
@@ -167,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             mbar_init(&bars[B_PFULL + t], 4);
             mbar_init(&bars[B_ODONE + t], 1);
         }
-        mbar_init(&bars[B_QFULL], 4);
+        mbar_init(&bars[B_QFULL], 8);
         mbar_init(&bars[B_DRAIN], 2);
         *abort_flag = 0;
         if (mt == 0 && kvh == 0 && n_words > p.max_words) set_status(p.d_status, LAZY_DSTATUS_BAD_TABLE);
@@ -183,6 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     tc::fence_after_sync();
     const uint32_t tbase = *tmem_slot;
 
+    if (warp < 4) {
+    setmaxnreg_dec<kProducerRegs>();
     if (warp == 0) {
         // ============================================================ table walk + K producer
         if (lane == 0) {
@@ -227,8 +252,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 // K tile
                 const int ks = j % kKStages;
                 if (!wait_or_abort(&bars[B_KEMPTY + ks], ((j / kKStages) & 1) ^ 1, abort_flag, p.d_status)) break;
-                mbar_arrive_expect_tx(&bars[B_KFULL + ks], n * kBlockBytes);
                 uint8_t *kd = sm + kOffK + ks * kTileBytes;
+                // blocks consecutive in the source: two 16 KiB boxes instead of 2n small ones
+                bool contig = true;
+#pragma unroll
+                for (int k = 1; k < kTileBlocks; ++k)
+                    contig = contig && (k >= n || word_block(wd[k]) == word_block(wd[0]) + static_cast<uint32_t>(k));
+                contig = PLAIN || (contig && word_block(wd[0]) < static_cast<uint32_t>(p.num_blocks) &&
+                                   word_block(wd[0]) + static_cast<uint32_t>(n) <= static_cast<uint32_t>(p.num_blocks));
+                if (contig) {
+                    mbar_arrive_expect_tx(&bars[B_KFULL + ks], 2 * kHalfPlane);
+                    const int z = PLAIN ? wbase + w : static_cast<int>(word_block(wd[0]));
+                    tma_load_4d(kd, &tmK8, 0, 0, kvh, z, &bars[B_KFULL + ks]);
+                    tma_load_4d(kd + kHalfPlane, &tmK8, kHalfDim, 0, kvh, z, &bars[B_KFULL + ks]);
+                } else {
+                mbar_arrive_expect_tx(&bars[B_KFULL + ks], n * kBlockBytes);
                 for (int k = 0; k < n; ++k) {
                     const uint32_t b = word_block(wd[k]);
                     int row;
@@ -240,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                     }
                     tma_load_2d(kd + k * kBoxBytes, &tmK, 0, row, &bars[B_KFULL + ks]);
                     tma_load_2d(kd + kHalfPlane + k * kBoxBytes, &tmK, kHalfDim, row, &bars[B_KFULL + ks]);
+                }
                 }
                 issued = j + 1;
                 w = wn;
@@ -262,14 +301,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 mbar_arrive(&bars[B_IEMPTY + is]);
                 const int vs = j % kVStages;
                 if (!wait_or_abort(&bars[B_VEMPTY + vs], ((j / kVStages) & 1) ^ 1, abort_flag, p.d_status)) break;
-                mbar_arrive_expect_tx(&bars[B_VFULL + vs], n * kBlockBytes);
                 uint8_t *vd = sm + kOffV + vs * kTileBytes;
+                bool contig = blk[0] < static_cast<uint32_t>(p.num_blocks) &&
+                              blk[0] + static_cast<uint32_t>(n) <= static_cast<uint32_t>(p.num_blocks);
+#pragma unroll
+                for (int k = 1; k < kTileBlocks; ++k) contig = contig && (k >= n || blk[k] == blk[0] + static_cast<uint32_t>(k));
+                if (contig) {
+                    mbar_arrive_expect_tx(&bars[B_VFULL + vs], 2 * kHalfPlane);
+                    tma_load_4d(vd, &tmV8, 0, 0, kvh, static_cast<int>(blk[0]), &bars[B_VFULL + vs]);
+                    tma_load_4d(vd + kHalfPlane, &tmV8, kHalfDim, 0, kvh, static_cast<int>(blk[0]), &bars[B_VFULL + vs]);
+                } else {
+                mbar_arrive_expect_tx(&bars[B_VFULL + vs], n * kBlockBytes);
                 for (int k = 0; k < n; ++k) {
                     const int row = blk[k] >= static_cast<uint32_t>(p.num_blocks)
                                         ? p.v_rows
                                         : (static_cast<int>(blk[k]) * p.hkv + kvh) * kBlockTokens;
                     tma_load_2d(vd + k * kBoxBytes, &tmV, 0, row, &bars[B_VFULL + vs]);
                     tma_load_2d(vd + kHalfPlane + k * kBoxBytes, &tmV, kHalfDim, row, &bars[B_VFULL + vs]);
+                }
                 }
                 issued = j + 1;
                 w += n;
@@ -330,8 +379,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             tc::commit(&bars[B_DRAIN]);
             mbar_wait(&bars[B_DRAIN], 0);
         }
-    } else if (warp >= 4 && warp < 12) {
+    }
+    } else if (warp < 12) {
         // ============================================================ softmax (one row per thread)
+        // The whole 128-column score row is held in registers: one tensor-memory load
+        // and one store (of P) per tile.
+        setmaxnreg_inc<kSoftmaxRegs>();
         const int t = (warp - 4) >> 2;                 // row tile
         const int row = threadIdx.x - 128 - 128 * t;   // 0..127 inside the tile
         const int R = R0 + kTileRows * t + row;
@@ -340,167 +393,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const int g = R % G;
         const int prow = pos0 + tok;
         const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-        const uint32_t tS = tbase + 128 * t, tO = tbase + 256 + 128 * t;
-        float m_run = -INFINITY, l_run = 0.f;
-        int j = 0;
-        bool ok = true;
-        for (int w = 0; w < n_words; ++j) {
-            const int is = j % kInfoStages;
-            if (!warp_wait(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) { ok = false; break; }
-            const TileInfo &ti = info[is];
-            const int n = ti.n, off = ti.off;
-            const bool full = (ti.flags & kFull) != 0;
-            int kj0[kTileBlocks], knv[kTileBlocks];
-#pragma unroll
-            for (int k = 0; k < kTileBlocks; ++k) {
-                kj0[k] = meta_j0(ti.meta[k]);
-                knv[k] = k < n ? meta_valid(ti.meta[k]) : 0;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_IEMPTY + is]);
-            if (!warp_wait(&bars[B_SFULL + t], j & 1, abort_flag, p.d_status)) { ok = false; break; }
-            tc::fence_after_sync();
-            // pass 1: masked row maximum (S_t(j) complete implies PV_t(j-1) complete).
-            // Two 32-column loads are in flight per wait.
-            float tmax = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 4; c += 2) {
-                uint32_t xa[32], xb[32];
-                tc::ld32(tS + lane_off + 32 * c, xa);
-                tc::ld32(tS + lane_off + 32 * (c + 1), xb);
-                tc::wait_ld();
-                if (full) {
-                    float m0 = __uint_as_float(xa[0]), m1 = __uint_as_float(xb[0]);
-#pragma unroll
-                    for (int e = 1; e < 32; ++e) {
-                        m0 = fmaxf(m0, __uint_as_float(xa[e]));
-                        m1 = fmaxf(m1, __uint_as_float(xb[e]));
-                    }
-                    tmax = fmaxf(tmax, fmaxf(m0, m1));
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) {
-                        const int col = 32 * c + e, k = col >> 4, si = col & 15;
-                        const uint32_t xv = e < 32 ? xa[e] : xb[e - 32];
-                        const bool vis = si < knv[k] && off + kj0[k] + si <= prow;
-                        tmax = vis ? fmaxf(tmax, __uint_as_float(xv)) : tmax;
-                    }
-                }
-            }
-            const float m_new = fmaxf(m_run, tmax);
-            const bool need = m_new > m_run + kRescaleThreshold;
-            float scale = 1.f;
-            if (need) {
-                scale = fast_exp2(m_run - m_new);
-                m_run = m_new;
-                l_run *= scale;
-            }
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t o[32];
-                    tc::ld32(tO + lane_off + 32 * c, o);
-                    tc::wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * scale);
-                    tc::st32(tO + lane_off + 32 * c, o);
-                }
-            }
-            const float mu = m_run == -INFINITY ? 0.f : m_run;
-            // pass 2: P = 2^(S - m) as bf16 pairs over the consumed S columns, row sum in fp32
-            float lsum = 0.f;
-#pragma unroll
-            for (int c = 0; c < 4; c += 2) {
-                uint32_t xa[32], xb[32];
-                tc::ld32(tS + lane_off + 32 * c, xa);
-                tc::ld32(tS + lane_off + 32 * (c + 1), xb);
-                tc::wait_ld();
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t *x = h == 0 ? xa : xb;
-                    const int cc = c + h;
-                    uint32_t pk[16];
-                    if (full) {
-                        float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const float p0 = fast_exp2(__uint_as_float(x[2 * e]) - mu);
-                            const float p1 = fast_exp2(__uint_as_float(x[2 * e + 1]) - mu);
-                            ls0 += p0;
-                            ls1 += p1;
-                            pk[e] = pack_bf16(p0, p1);
-                        }
-                        lsum += ls0 + ls1;
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            float pr[2];
-#pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                const int col = 32 * cc + 2 * e + hh, k = col >> 4, si = col & 15;
-                                const bool vis = si < knv[k] && off + kj0[k] + si <= prow;
-                                pr[hh] = vis ? fast_exp2(__uint_as_float(x[2 * e + hh]) - mu) : 0.f;
-                            }
-                            lsum += pr[0] + pr[1];
-                            pk[e] = pack_bf16(pr[0], pr[1]);
-                        }
-                    }
-                    // P columns 16cc..16cc+15 were S columns already read in this or an earlier chunk
-                    tc::st16(tS + lane_off + 16 * cc, pk);
-                }
-            }
-            l_run += lsum;
-            tc::wait_st();
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_PFULL + t]);
-            w += n;
-        }
-        // ------------------------------------------------------------ epilogue
-        bool have = ok && j > 0;
-        if (have) have = warp_wait(&bars[B_ODONE + t], (j - 1) & 1, abort_flag, p.d_status);
-        const float inv = (have && l_run > 0.f) ? 1.f / l_run : 0.f;
-        const bool all_have = __all_sync(0xffffffffu, have);
-        if (all_have) tc::fence_after_sync();
-        uint4 *o = row_ok ? reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(q0 + tok) * p.hq + kvh * G + g) *
-                                                                  kHeadDim)
-                          : nullptr;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint32_t ob[32];
-            if (all_have) {
-                tc::ld32(tO + lane_off + 32 * c, ob);
-                tc::wait_ld();
-            } else {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) ob[e] = 0u;
-            }
-            if (o) {
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    uint4 u;
-                    u.x = pack_bf16(__uint_as_float(ob[8 * v + 0]) * inv, __uint_as_float(ob[8 * v + 1]) * inv);
-                    u.y = pack_bf16(__uint_as_float(ob[8 * v + 2]) * inv, __uint_as_float(ob[8 * v + 3]) * inv);
-                    u.z = pack_bf16(__uint_as_float(ob[8 * v + 4]) * inv, __uint_as_float(ob[8 * v + 5]) * inv);
-                    u.w = pack_bf16(__uint_as_float(ob[8 * v + 6]) * inv, __uint_as_float(ob[8 * v + 7]) * inv);
-                    o[4 * c + v] = u;
-                }
-            }
-        }
-    } else if (warp >= 12) {
-        // ============================================================ rotations
-        // (1) Q'_i = R(p_i - P0) q_i once per CTA (R(p_i) on the plain path), P0 =
-        //     the CTA's first query position.  Thread (ch, rb) writes pairs
-        //     8ch..8ch+7 of rows rb + 16k of each row tile; between rows rb + 16k
-        //     and rb + 16(k+1) the token advances by dlo = 16 / G or dlo + 1
-        //     tokens, so angles advance by rotation with two step tables.
-        // (2) lazy path only: every K tile, once TMA has landed it, is rotated
-        //     in shared memory by (o - P0) -- one relative rotation per tile --
-        //     so that scores carry the angle (p_i - o - j).
-        const int tid = threadIdx.x - 384;
-        const int ch = tid & 7;
-        const int rb = tid >> 3;
+        // Q'_i = R(p_i - P0) q_i for this warpgroup's row tile (R(p_i) on the plain path):
+        // thread (ch, rb) writes pairs 8ch..8ch+7 of rows rb + 16k; between rows rb + 16k and
+        // rb + 16(k+1) the token advances by dlo = 16 / G or dlo + 1, so the angles advance by
+        // rotations from two step tables.
         {
+            const int ch = row & 7, rb = row >> 3;
             const int dlo = 16 / G;
             float cA[8], sA[8], cB[8], sB[8];
 #pragma unroll
@@ -509,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 rope_cos_sin(dlo + 1, theta_s[8 * ch + e], cB[e], sB[e]);
             }
             const int qref = PLAIN ? 0 : Pbase;
-            for (int t = 0; t < 2; ++t) {
+            {
                 const int rowbase = R0 + kTileRows * t + rb;   // global row of k = 0
                 int tk_prev = rowbase / G;
                 float cc[8], ss[8];
@@ -572,6 +470,125 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_QFULL]);
         }
+        const uint32_t tS = tbase + 128 * t, tO = tbase + 256 + 128 * t;
+        float m_run = -INFINITY, l_run = 0.f;
+        int j = 0;
+        bool ok = true;
+        for (int w = 0; w < n_words; ++j) {
+            const int is = j % kInfoStages;
+            if (!warp_wait(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) { ok = false; break; }
+            const TileInfo &ti = info[is];
+            const int n = ti.n;
+            const bool full = (ti.flags & kFull) != 0;
+            // visible keys of each 16-key block for this row: slots si < lim[k]
+            int lim[kTileBlocks];
+#pragma unroll
+            for (int k = 0; k < kTileBlocks; ++k) {
+                const int nv = k < n ? meta_valid(ti.meta[k]) : 0;
+                lim[k] = max(0, min(nv, prow - ti.off - meta_j0(ti.meta[k]) + 1));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[B_IEMPTY + is]);
+            if (!warp_wait(&bars[B_SFULL + t], j & 1, abort_flag, p.d_status)) { ok = false; break; }
+            tc::fence_after_sync();
+            // S_t(j) complete implies PV_t(j-1) complete
+            uint32_t sv[128];
+            tc::ld32(tS + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(sv + 0));
+            tc::ld32(tS + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+            tc::ld32(tS + lane_off + 64, *reinterpret_cast<uint32_t(*)[32]>(sv + 64));
+            tc::ld32(tS + lane_off + 96, *reinterpret_cast<uint32_t(*)[32]>(sv + 96));
+            tc::wait_ld();
+            if (!full) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    sv[c] = (c & 15) < lim[c >> 4] ? sv[c] : 0xFF800000u;   // -inf: P = 0
+            }
+            float m0 = __uint_as_float(sv[0]), m1 = __uint_as_float(sv[1]);
+#pragma unroll
+            for (int c = 2; c < 128; c += 2) {
+                m0 = fmaxf(m0, __uint_as_float(sv[c]));
+                m1 = fmaxf(m1, __uint_as_float(sv[c + 1]));
+            }
+            const float m_new = fmaxf(m_run, fmaxf(m0, m1));
+            const bool need = m_new > m_run + kRescaleThreshold;
+            float scale = 1.f;
+            if (need) {
+                scale = fast_exp2(m_run - m_new);
+                m_run = m_new;
+                l_run *= scale;
+            }
+            const float mu = m_run == -INFINITY ? 0.f : m_run;
+            // P = 2^(S - m) as bf16 pairs over the first 64 columns of S, row sum in fp32
+            float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+            for (int e = 0; e < 64; ++e) {
+                const float p0 = fast_exp2(__uint_as_float(sv[2 * e]) - mu);
+                const float p1 = fast_exp2(__uint_as_float(sv[2 * e + 1]) - mu);
+                ls0 += p0;
+                ls1 += p1;
+                sv[e] = pack_bf16(p0, p1);
+            }
+            tc::st32(tS + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(sv + 0));
+            tc::st32(tS + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+            l_run += ls0 + ls1;
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tc::ld32(tO + lane_off + 32 * c, o);
+                    tc::wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * scale);
+                    tc::st32(tO + lane_off + 32 * c, o);
+                }
+            }
+            tc::wait_st();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[B_PFULL + t]);
+            w += n;
+        }
+        // ------------------------------------------------------------ epilogue
+        bool have = ok && j > 0;
+        if (have) have = warp_wait(&bars[B_ODONE + t], (j - 1) & 1, abort_flag, p.d_status);
+        const float inv = (have && l_run > 0.f) ? 1.f / l_run : 0.f;
+        const bool all_have = __all_sync(0xffffffffu, have);
+        if (all_have) tc::fence_after_sync();
+        uint4 *o = row_ok ? reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(q0 + tok) * p.hq + kvh * G + g) *
+                                                                  kHeadDim)
+                          : nullptr;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t ob[32];
+            if (all_have) {
+                tc::ld32(tO + lane_off + 32 * c, ob);
+                tc::wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) ob[e] = 0u;
+            }
+            if (o) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    uint4 u;
+                    u.x = pack_bf16(__uint_as_float(ob[8 * v + 0]) * inv, __uint_as_float(ob[8 * v + 1]) * inv);
+                    u.y = pack_bf16(__uint_as_float(ob[8 * v + 2]) * inv, __uint_as_float(ob[8 * v + 3]) * inv);
+                    u.z = pack_bf16(__uint_as_float(ob[8 * v + 4]) * inv, __uint_as_float(ob[8 * v + 5]) * inv);
+                    u.w = pack_bf16(__uint_as_float(ob[8 * v + 6]) * inv, __uint_as_float(ob[8 * v + 7]) * inv);
+                    o[4 * c + v] = u;
+                }
+            }
+        }
+    } else {
+        // ============================================================ rotations
+        setmaxnreg_dec<kRotRegs>();
+        // Lazy path only: every K tile, once TMA has landed it, is rotated in
+        // shared memory by (o - P0) -- one relative rotation per tile -- so that
+        // scores carry the angle (p_i - o - j).  Thread (ch, rb) handles pairs
+        // 8ch..8ch+7 of key rows rb + 16k.
+        const int tid = threadIdx.x - 384;
+        const int ch = tid & 7;
+        const int rb = tid >> 3;
         if (!PLAIN) {
             int cur = INT_MIN;
             float kc[8], kn[8];
@@ -633,21 +650,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 }
 
 template <bool PLAIN>
-cudaError_t launch_t(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, cudaStream_t s) {
+cudaError_t launch_t(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8, const CUtensorMap &tv8,
+                     const AttnParams &p, cudaStream_t s) {
     auto kern = prefill_tc_kernel<PLAIN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
     if (e != cudaSuccess) return e;
     const int mtiles = (p.max_q * p.group + kRows - 1) / kRows;
     dim3 grid(max(1, mtiles), p.hkv, p.num_req);
-    kern<<<grid, kThreads, kTcSmem, s>>>(tk, tv, p);
+    kern<<<grid, kThreads, kTcSmem, s>>>(tk, tv, tk8, tv8, p);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_prefill_tc(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, bool plain,
-                              cudaStream_t s) {
-    return plain ? launch_t<true>(tk, tv, p, s) : launch_t<false>(tk, tv, p, s);
+cudaError_t launch_prefill_tc(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8,
+                              const CUtensorMap &tv8, const AttnParams &p, bool plain, cudaStream_t s) {
+    return plain ? launch_t<true>(tk, tv, tk8, tv8, p, s) : launch_t<false>(tk, tv, tk8, tv8, p, s);
 }
 
 }  // namespace lazy
