@@ -564,6 +564,25 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args):
+    """A small case for profiler captures: 2 prefill requests (64 CTAs) or 8 decode requests of the
+    8B shapes over a 100-document pool, the attention kernel launched --steps times."""
+    import torch
+    from position_agnostic_paged_b200 import workloads as W
+    from position_agnostic_paged_b200.runner import DevicePool, DeviceStep
+    if args.profile_case == "prefill_small":
+        wl = W.make("prefill_8b", n_docs=100, n_prefill=2)
+    else:
+        wl = W.make("decode_8b", n_docs=100, n_decode=8)
+    pool = DevicePool(wl).setup()
+    ds = DeviceStep(pool, wl.steps[0])
+    ds.write_new_tokens()
+    for _ in range(args.steps):
+        ds.attend()
+    torch.cuda.synchronize()
+    log(f"[profile-case] {args.profile_case}: {args.steps} launches, status {pool.status()}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -577,12 +596,17 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--extended", action="store_true",
                     help="also time decode 70B (Zipf 1.2 and uniform) and the mixed 8B step (GQA, MQA)")
+    ap.add_argument("--profile-case", choices=["prefill_small", "decode_small"],
+                    help="launch only the attention kernel of a small case --steps times (for ncu captures; "
+                         "prints no result line)")
     ap.add_argument("--cpu-requests", type=int, default=64)
     ap.add_argument("--ref-requests", type=int, default=2)
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.profile_case:
+        run_profile_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -4,7 +4,9 @@ Each distinct source range of the case's token store becomes one document
 stored once in the paged pool (its tokens at local indices 0..len-1); every
 segment that uses it becomes table words (block, offset).  Two segments with
 the same source therefore share one physical copy, as in the pages' zero-copy
-reuse.
+reuse.  By default a document's blocks are consecutive in the pool; with
+`scatter_seed` they are placed by a seeded permutation of the pool's blocks, so
+that runs of a tile's blocks are (mostly) not consecutive.
 """
 from __future__ import annotations
 
@@ -23,7 +25,7 @@ def _i32(a, dev):
 
 
 class DeviceCase:
-    def __init__(self, case, dev="cuda", extra_blocks: int = 0):
+    def __init__(self, case, dev="cuda", extra_blocks: int = 0, scatter_seed: int | None = None):
         self.case = case
         self.cfg = la.Cfg(case.hq, case.hkv, rope_base=case.base)
         docs = {}
@@ -37,6 +39,11 @@ class DeviceCase:
             self.doc_block[src] = nb
             nb += (docs[src] + 15) // 16
         self.num_blocks = nb + extra_blocks
+        # logical block (document-major) -> physical block of the pool
+        if scatter_seed is None:
+            self.phys = np.arange(max(self.num_blocks, 1))
+        else:
+            self.phys = np.random.default_rng(scatter_seed).permutation(max(self.num_blocks, 1))
         shape = (max(self.num_blocks, 1), case.hkv, 16, case.d)
         self.k_pool = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
         self.v_pool = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
@@ -46,7 +53,7 @@ class DeviceCase:
         for src, ln in docs.items():
             for j in range(ln):
                 rows.append(src + j)
-                slots.append(self.doc_block[src] * 16 + j)
+                slots.append(int(self.phys[self.doc_block[src] + j // 16]) * 16 + j % 16)
                 js.append(j)
         if rows:
             la.kv_write(self.cfg, _u16(case.k_tok[rows], dev), _u16(case.v_tok[rows], dev), _i32(slots, dev),
@@ -56,7 +63,7 @@ class DeviceCase:
             for g in range(case.seg_indptr[r], case.seg_indptr[r + 1]):
                 src, off, ln = int(case.seg_src[g]), int(case.seg_off[g]), int(case.seg_len[g])
                 for k in range((ln + 15) // 16):
-                    blocks.append(self.doc_block[src] + k)
+                    blocks.append(int(self.phys[self.doc_block[src] + k]))
                     offs.append(off)
             indptr.append(len(blocks))
         self.words = la.pack_words(np.array(blocks, np.int32), np.array(offs, np.int32))

@@ -172,6 +172,32 @@ def test_adversarial_cases_all_group_sizes(kind, hq, hkv):
     assert dc.status() == 0
 
 
+# ----------------------------------------------------------------------------- block placement
+def _long_requests(decode: bool):
+    # documents of 200 and 130 tokens (full 8-block tiles and partial ones), one of
+    # them reused at two offsets
+    segs = [(0, 0, 200), (300, 210, 130), (0, 400, 200)]
+    if decode:
+        return [(segs, [700]), ([(300, 0, 130)], [140])]
+    return [(segs, list(range(600, 700))), ([(300, 0, 130)], list(range(130, 190)))]
+
+
+@pytest.mark.parametrize("scatter", [None, 7])
+@pytest.mark.parametrize("kind", ["decode", "prefill"])
+def test_scattered_document_blocks(kind, scatter):
+    """A document's blocks need not be consecutive in the pool: tiles whose blocks
+    are scattered take the per-block load path and give the same results."""
+    case = make_case(31, hq=32, hkv=8, d=128, requests=_long_requests(kind == "decode"))
+    dc = DeviceCase(case, scatter_seed=scatter)
+    ref = oracle.attend(**case.oracle_kwargs())
+    tol = edge_max_abs(case)
+    got = dc.decode() if kind == "decode" else dc.prefill()
+    check(got, ref, max_abs=tol, what=f"{kind} scatter={scatter} lazy")
+    got_p = dc.decode(plain=True) if kind == "decode" else dc.prefill(plain=True)
+    check(got_p, ref, max_abs=tol, what=f"{kind} scatter={scatter} plain")
+    assert dc.status() == 0
+
+
 def test_queries_that_see_nothing_give_zero_rows():
     case = make_case(5, hq=8, hkv=2, d=128, requests=[([(0, 100, 20)], [50]), ([(20, 0, 16)], [15])])
     dc = DeviceCase(case)
