@@ -50,7 +50,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch of the dominant kernels from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
 # kernel source it was taken on; reported as null when the source changed.
-TRAFFIC = {}
+TRAFFIC = {
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
+    #     -k regex:decode_split -s 3 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu --no-compare --no-e2e
+    "decode_8b": {"sha": "1882d73735d88144", "bytes": 782188544 + 7172352},
+    # the same with -k regex:prefill_tc
+    "prefill_8b": {"sha": "19cfa1b7f0e3a1be", "bytes": 302290432 + 27631616},
+}
 
 
 def log(*a):

@@ -187,9 +187,6 @@ int prefill_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t 
         !make_blocks_map(&tv8, v_pool, num_blocks, p.hkv))
         return LAZY_ECUDA;
     // each request writes exactly its own query tokens' rows
-    const char *impl = getenv("LAZY_ATTN_PREFILL_IMPL");
-    if (impl && impl[0] == 'm')
-        return launch_rc(launch_prefill(tk, tv, p, plain, static_cast<cudaStream_t>(stream)));
     return launch_rc(launch_prefill_tc(tk, tv, tk8, tv8, p, plain, static_cast<cudaStream_t>(stream)));
 }
 

@@ -75,8 +75,6 @@ cudaError_t launch_decode_table(const DecodeTableParams &p, cudaStream_t s);
 cudaError_t launch_materialize(const MaterializeParams &p, cudaStream_t s);
 cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, bool plain,
                           cudaStream_t s);
-cudaError_t launch_prefill(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, bool plain,
-                           cudaStream_t s);
 // tk, tv: the K source and V pool as rows of 128 bf16 (one box = half of one block);
 // tk8, tv8: the same memory as (d, token, head, block) (one box = half of 8 consecutive blocks).
 cudaError_t launch_prefill_tc(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8,
