@@ -165,7 +165,15 @@ int lazy_decode_attn_noalloc(const lazy_attn_cfg *cfg, const uint16_t *q_raw, co
 /* Bytes of the built-in scratch array used by lazy_decode_attn_noalloc. */
 size_t lazy_decode_noalloc_capacity(void);
 
-/* Workspace for lazy_prefill_attn. */
+/* Workspace for lazy_prefill_attn on the current device.  The prefill work is
+ * one unit per 256 query rows of one KV head of one request, one CTA per SM;
+ * when the last wave of units would leave at least half of the SMs idle, each
+ * of its units runs as two CTAs over the two halves of the request's table
+ * words, and their partial results (fp32 O, running max and sum per row) are
+ * merged by a second kernel.  This returns the bytes those partial results
+ * need (0 when no unit is split); lazy_prefill_attn balances the last wave
+ * only when given at least that much workspace, and runs unsplit otherwise.
+ * The result does not depend on the split beyond fp32 rounding order. */
 size_t lazy_prefill_workspace_bytes(const lazy_attn_cfg *cfg, int num_req, int total_q, int max_q,
                                     int max_words);
 

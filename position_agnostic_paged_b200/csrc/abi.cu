@@ -66,6 +66,14 @@ bool make_blocks_map(CUtensorMap *map, const void *base, int64_t nblocks, int hk
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Streaming multiprocessors of the current device (0 if it cannot be queried).
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
 int check_cfg(const lazy_attn_cfg *cfg) {
     if (!cfg) return LAZY_EINVAL;
     if (cfg->head_dim != 128 || cfg->block_size != 16) return LAZY_ESHAPE;
@@ -179,6 +187,16 @@ int prefill_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t 
     p.cu_q = cu_q;
     p.q_pos0 = q_pos0;
     p.max_q = max_q;
+    // work units and, with a large enough workspace, the split of the last partial wave
+    p.pf_mtiles = static_cast<int>((static_cast<int64_t>(max_q) * p.group + kPrefillRows - 1) / kPrefillRows);
+    const long long units = static_cast<long long>(p.pf_mtiles) * p.hkv * num_req;
+    if (units > (1LL << 30)) return LAZY_ERANGE;
+    int nsplit = prefill_split_units(units, sm_count());
+    if (!workspace || ws_bytes < prefill_split_bytes(nsplit)) nsplit = 0;
+    p.pf_nsplit = nsplit;
+    p.pf_base = static_cast<int>(units) - nsplit;
+    p.ws_acc = static_cast<float *>(workspace);
+    p.ws_ml = nsplit ? p.ws_acc + static_cast<size_t>(nsplit) * 2 * kPrefillRows * 128 : nullptr;
     p.k_rows = static_cast<int>(k_rows);
     p.v_rows = static_cast<int>(static_cast<int64_t>(num_blocks) * p.hkv * 16);
     CUtensorMap tk, tv, tk8, tv8;
@@ -260,12 +278,12 @@ int lazy_decode_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int3
 }
 
 size_t lazy_prefill_workspace_bytes(const lazy_attn_cfg *cfg, int num_req, int total_q, int max_q, int max_words) {
-    (void)cfg;
-    (void)num_req;
     (void)total_q;
-    (void)max_q;
     (void)max_words;
-    return 0;
+    if (!cfg || check_cfg(cfg) != LAZY_OK || num_req <= 0 || max_q <= 0) return 0;
+    const int G = cfg->num_q_heads / cfg->num_kv_heads;
+    const long long mtiles = (static_cast<long long>(max_q) * G + kPrefillRows - 1) / kPrefillRows;
+    return prefill_split_bytes(prefill_split_units(mtiles * cfg->num_kv_heads * num_req, sm_count()));
 }
 
 int lazy_prefill_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *cu_q, const int32_t *q_pos0,

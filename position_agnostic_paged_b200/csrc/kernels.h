@@ -58,6 +58,11 @@ struct AttnParams {
     int num_req, hq, hkv, group, num_blocks, max_words;
     int words_per_split, n_splits;   // decode
     int max_q;                       // prefill
+    // prefill work split: units (m-tile, KV head, request) in the order of a 3D grid
+    // (m-tile fastest); units below pf_base run whole, the pf_nsplit units from pf_base run as
+    // two CTAs each over the first and second half of the table's words, writing partial
+    // results to ws_acc / ws_ml that prefill_combine merges
+    int pf_mtiles, pf_base, pf_nsplit;
     int k_rows, v_rows;              // rows (of 128 bf16) covered by the K and V tensor maps
     float scale_log2;            // softmax scale * log2(e)
     RopeTableHost rope;
@@ -79,5 +84,16 @@ cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const At
 // tk8, tv8: the same memory as (d, token, head, block) (one box = half of 8 consecutive blocks).
 cudaError_t launch_prefill_tc(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8,
                               const CUtensorMap &tv8, const AttnParams &p, bool plain, cudaStream_t s);
+constexpr int kPrefillRows = 256;   // query rows per prefill CTA
+// Units of the last, partial wave that are split in two when that wave is at most half full
+// (one prefill CTA per SM): the grid then ends with two half-length CTAs per such unit.
+inline int prefill_split_units(long long units, int sms) {
+    if (units <= 0 || sms <= 0) return 0;
+    const long long rem = units % sms;
+    return (rem > 0 && 2 * rem <= sms) ? static_cast<int>(rem) : 0;
+}
+inline size_t prefill_split_bytes(int nsplit) {
+    return static_cast<size_t>(nsplit) * 2 * kPrefillRows * (128 + 2) * sizeof(float);
+}
 
 }  // namespace lazy

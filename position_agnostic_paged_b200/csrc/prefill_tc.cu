@@ -156,7 +156,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);
 
-    const int mt = blockIdx.x, kvh = blockIdx.y, r = blockIdx.z;
+    // work unit (m-tile, KV head, request) and which part of its keys this CTA takes
+    int unit = static_cast<int>(blockIdx.x), part = -1;
+    if (unit >= p.pf_base) {
+        const int k = unit - p.pf_base;
+        unit = p.pf_base + (k >> 1);
+        part = k & 1;
+    }
+    const int mt = unit % p.pf_mtiles, kvh = (unit / p.pf_mtiles) % p.hkv, r = unit / (p.pf_mtiles * p.hkv);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.group;
     const int q0 = p.cu_q[r];
@@ -165,6 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     if (R0 >= T * G) return;   // uniform: this tile has no rows
     const int wbase = p.table_indptr[r];
     const int n_words = p.table_indptr[r + 1] - wbase;
+    // words this CTA walks: all of them, or the first or second half for a split unit
+    const int wbeg = part == 1 ? n_words / 2 : 0, wend = part == 0 ? n_words / 2 : n_words;
     const uint32_t *tbl = p.table + wbase;
     const int pos0 = p.q_pos0[r];
     const int tok_first = R0 / G;
@@ -213,16 +222,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         if (lane == 0) {
             tma_prefetch_desc(&tmK);
             int issued = 0;
-            for (int w = 0, j = 0; w < n_words; ++j) {
+            for (int w = wbeg, j = 0; w < wend; ++j) {
                 // the tile: up to 8 consecutive words that share one offset
                 uint32_t wd[kTileBlocks];
 #pragma unroll
-                for (int k = 0; k < kTileBlocks; ++k) wd[k] = (w + k < n_words) ? tbl[w + k] : 0xFFFFFFFFu;
+                for (int k = 0; k < kTileBlocks; ++k) wd[k] = (w + k < wend) ? tbl[w + k] : 0xFFFFFFFFu;
                 const int off = word_offset(wd[0]);
                 int n = 1;
 #pragma unroll
                 for (int k = 1; k < kTileBlocks; ++k)
-                    if (n == k && w + k < n_words && word_offset(wd[k]) == off) n = k + 1;
+                    if (n == k && w + k < wend && word_offset(wd[k]) == off) n = k + 1;
                 const int wn = w + n;
                 uint32_t mt_k[kTileBlocks];
                 bool full = n == kTileBlocks;
@@ -291,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         if (lane == 0) {
             tma_prefetch_desc(&tmV);
             int issued = 0;
-            for (int w = 0, j = 0; w < n_words; ++j) {
+            for (int w = wbeg, j = 0; w < wend; ++j) {
                 const int is = j % kInfoStages;
                 if (!wait_or_abort(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) break;
                 const int n = info[is].n;
@@ -344,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             const uint64_t dQ = tc::smem_desc(sQ + t * kTileBytes, 16, 1024), dK0 = tc::smem_desc(sK, 16, 1024);
             const uint64_t dV0 = tc::smem_desc(sV, kHalfPlane, 1024);
             bool ok = wait_or_abort(&bars[B_QFULL], 0, abort_flag, p.d_status);
-            for (int w = 0, j = 0; w < n_words && ok; ++j) {
+            for (int w = wbeg, j = 0; w < wend && ok; ++j) {
                 const int is = j % kInfoStages;
                 if (!wait_or_abort(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) break;
                 const int n = info[is].n;
@@ -474,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         float m_run = -INFINITY, l_run = 0.f;
         int j = 0;
         bool ok = true;
-        for (int w = 0; w < n_words; ++j) {
+        for (int w = wbeg; w < wend; ++j) {
             const int is = j % kInfoStages;
             if (!warp_wait(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) { ok = false; break; }
             const TileInfo &ti = info[is];
@@ -554,11 +563,34 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const float inv = (have && l_run > 0.f) ? 1.f / l_run : 0.f;
         const bool all_have = __all_sync(0xffffffffu, have);
         if (all_have) tc::fence_after_sync();
-        uint4 *o = row_ok ? reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(q0 + tok) * p.hq + kvh * G + g) *
-                                                                  kHeadDim)
-                          : nullptr;
+        if (part >= 0) {
+            // half of a split unit: unnormalised O, running max and sum (log2 domain) for the
+            // combine step
+            const size_t srow = static_cast<size_t>((unit - p.pf_base) * 2 + part) * kRows + kTileRows * t + row;
+            float4 *wo = reinterpret_cast<float4 *>(p.ws_acc + srow * kHeadDim);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 4; ++c) {
+                uint32_t ob[32];
+                if (all_have) {
+                    tc::ld32(tO + lane_off + 32 * c, ob);
+                    tc::wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) ob[e] = 0u;
+                }
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                    wo[8 * c + v] = make_float4(__uint_as_float(ob[4 * v]), __uint_as_float(ob[4 * v + 1]),
+                                                __uint_as_float(ob[4 * v + 2]), __uint_as_float(ob[4 * v + 3]));
+            }
+            p.ws_ml[2 * srow] = have ? m_run : -INFINITY;
+            p.ws_ml[2 * srow + 1] = have ? l_run : 0.f;
+        }
+        uint4 *o = (row_ok && part < 0) ? reinterpret_cast<uint4 *>(p.out + (static_cast<size_t>(q0 + tok) * p.hq +
+                                                                              kvh * G + g) * kHeadDim)
+                                        : nullptr;
+#pragma unroll
+        for (int c = 0; c < 4 && part < 0; ++c) {
             uint32_t ob[32];
             if (all_have) {
                 tc::ld32(tO + lane_off + 32 * c, ob);
@@ -592,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         if (!PLAIN) {
             int cur = INT_MIN;
             float kc[8], kn[8];
-            for (int w = 0, j = 0; w < n_words; ++j) {
+            for (int w = wbeg, j = 0; w < wend; ++j) {
                 const int is = j % kInfoStages;
                 bool okw = wait_or_abort(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status);
                 if (!rot_all(okw)) break;
@@ -649,15 +681,43 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     }
 }
 
+// Merges the two halves of each split unit: with M = max(m0, m1) and w_i = 2^(m_i - M),
+// O = (w0 O0 + w1 O1) / (w0 l0 + w1 l1) -- the same merge as between consecutive key tiles
+// of one CTA.  One warp per query row, 4 columns of d per lane.
+__global__ void __launch_bounds__(256) prefill_combine_kernel(const AttnParams p) {
+    const int s = blockIdx.x, row_in = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    const int unit = p.pf_base + s;
+    const int mt = unit % p.pf_mtiles, kvh = (unit / p.pf_mtiles) % p.hkv, r = unit / (p.pf_mtiles * p.hkv);
+    const int G = p.group;
+    const int q0 = p.cu_q[r], T = p.cu_q[r + 1] - q0;
+    const int R = mt * kRows + row_in;
+    if (R >= T * G) return;
+    const size_t r0 = static_cast<size_t>(2 * s) * kRows + row_in, r1 = r0 + kRows;
+    const float m0 = p.ws_ml[2 * r0], l0 = p.ws_ml[2 * r0 + 1], m1 = p.ws_ml[2 * r1], l1 = p.ws_ml[2 * r1 + 1];
+    const float M = fmaxf(m0, m1);
+    const float w0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M), w1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
+    const float L = w0 * l0 + w1 * l1;
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    const float4 a = reinterpret_cast<const float4 *>(p.ws_acc + r0 * kHeadDim)[lane];
+    const float4 b = reinterpret_cast<const float4 *>(p.ws_acc + r1 * kHeadDim)[lane];
+    uint2 u;
+    u.x = pack_bf16((w0 * a.x + w1 * b.x) * inv, (w0 * a.y + w1 * b.y) * inv);
+    u.y = pack_bf16((w0 * a.z + w1 * b.z) * inv, (w0 * a.w + w1 * b.w) * inv);
+    const int tok = R / G, g = R % G;
+    reinterpret_cast<uint2 *>(p.out + (static_cast<size_t>(q0 + tok) * p.hq + kvh * G + g) * kHeadDim)[lane] = u;
+}
+
 template <bool PLAIN>
 cudaError_t launch_t(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8, const CUtensorMap &tv8,
                      const AttnParams &p, cudaStream_t s) {
     auto kern = prefill_tc_kernel<PLAIN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
     if (e != cudaSuccess) return e;
-    const int mtiles = (p.max_q * p.group + kRows - 1) / kRows;
-    dim3 grid(max(1, mtiles), p.hkv, p.num_req);
-    kern<<<grid, kThreads, kTcSmem, s>>>(tk, tv, tk8, tv8, p);
+    static_assert(kRows == kPrefillRows, "rows per CTA");
+    kern<<<p.pf_base + 2 * p.pf_nsplit, kThreads, kTcSmem, s>>>(tk, tv, tk8, tv8, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.pf_nsplit == 0) return e;
+    prefill_combine_kernel<<<dim3(p.pf_nsplit, kRows / 8), 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 

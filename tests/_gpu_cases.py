@@ -91,7 +91,9 @@ class DeviceCase:
                            self.k_pool, self.v_pool, out, ws, self.d_status)
         return out.float().cpu().numpy().astype(np.float64).reshape(-1, c.d)
 
-    def prefill(self, plain: bool = False):
+    def prefill(self, plain: bool = False, split: bool = True):
+        """split: pass the workspace lazy_prefill_workspace_bytes asks for, so that the units of
+        a partial last wave run as two halves merged by the combine kernel."""
         c = self.case
         n = c.cu_q.size - 1
         q_pos0 = []
@@ -105,14 +107,18 @@ class DeviceCase:
         q = _u16(c.q_raw, self.dev)
         cu = _i32(c.cu_q, self.dev)
         p0 = _i32(q_pos0, self.dev)
+        ws = None
+        if split:
+            nb = la.prefill_workspace_bytes(self.cfg, n, total_q, max_q, self.max_words)
+            ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=self.dev)
         if plain:
             kmat = torch.empty((self.table.numel(), c.hkv, 16, c.d), dtype=torch.bfloat16, device=self.dev)
             la.materialize_k(self.cfg, self.table, self.blk_meta, self.k_pool, kmat, self.d_status)
             la.plain_prefill_attn(self.cfg, q, cu, p0, max_q, self.table, self.table_indptr, self.max_words,
-                                  self.blk_meta, kmat, self.v_pool, out, None, self.d_status)
+                                  self.blk_meta, kmat, self.v_pool, out, ws, self.d_status)
         else:
             la.prefill_attn(self.cfg, q, cu, p0, max_q, self.table, self.table_indptr, self.max_words,
-                            self.blk_meta, self.k_pool, self.v_pool, out, None, self.d_status)
+                            self.blk_meta, self.k_pool, self.v_pool, out, ws, self.d_status)
         return out.float().cpu().numpy().astype(np.float64).reshape(-1, c.d)
 
     def status(self) -> int:

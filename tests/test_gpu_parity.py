@@ -159,15 +159,18 @@ def _adv_requests(decode: bool):
 
 
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 2), (32, 8), (64, 8), (32, 1), (16, 1)])
-@pytest.mark.parametrize("kind", ["decode", "prefill"])
+@pytest.mark.parametrize("kind", ["decode", "prefill", "prefill_unsplit"])
 def test_adversarial_cases_all_group_sizes(kind, hq, hkv):
+    """prefill: every unit runs as two halves merged by the combine kernel (small batches leave
+    most SMs idle); prefill_unsplit: no workspace, one CTA per unit."""
     case = make_case(100 + hq + hkv, hq=hq, hkv=hkv, d=128, requests=_adv_requests(kind == "decode"))
     dc = DeviceCase(case)
     ref = oracle.attend(**case.oracle_kwargs())
     tol = edge_max_abs(case)
-    got = dc.decode() if kind == "decode" else dc.prefill()
+    split = kind == "prefill"
+    got = dc.decode() if kind == "decode" else dc.prefill(split=split)
     check(got, ref, max_abs=tol, what=f"{kind} G={hq // hkv} lazy")
-    got_p = dc.decode(plain=True) if kind == "decode" else dc.prefill(plain=True)
+    got_p = dc.decode(plain=True) if kind == "decode" else dc.prefill(plain=True, split=split)
     check(got_p, ref, max_abs=tol, what=f"{kind} G={hq // hkv} plain")
     assert dc.status() == 0
 
