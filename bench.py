@@ -572,16 +572,20 @@ def run_reference(args):
 
 def run_profile_case(args):
     """A small case for profiler captures: 2 prefill requests (64 CTAs) or 8 decode requests of the
-    8B shapes over a 100-document pool, the attention kernel launched --steps times."""
+    8B shapes over a 100-document pool, or 32 decode requests of the MQA shapes (Hq 32, Hkv 1) over
+    a 400-document pool; the attention kernel launched --steps times."""
     import torch
     from position_agnostic_paged_b200 import workloads as W
     from position_agnostic_paged_b200.runner import DevicePool, DeviceStep
     if args.profile_case == "prefill_small":
         wl = W.make("prefill_8b", n_docs=100, n_prefill=2)
-    else:
+    elif args.profile_case == "decode_small":
         wl = W.make("decode_8b", n_docs=100, n_decode=8)
+    else:
+        wl = W.make("mixed_8b_mqa", n_docs=400, n_prefill=0, n_decode=32)
     pool = DevicePool(wl).setup()
-    ds = DeviceStep(pool, wl.steps[0])
+    ds = DeviceStep(pool, [st for st in wl.steps if st.kind == ("prefill" if "prefill" in args.profile_case
+                                                                    else "decode")][0])
     ds.write_new_tokens()
     for _ in range(args.steps):
         ds.attend()
@@ -602,7 +606,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--extended", action="store_true",
                     help="also time decode 70B (Zipf 1.2 and uniform) and the mixed 8B step (GQA, MQA)")
-    ap.add_argument("--profile-case", choices=["prefill_small", "decode_small"],
+    ap.add_argument("--profile-case", choices=["prefill_small", "decode_small", "decode_mqa_small"],
                     help="launch only the attention kernel of a small case --steps times (for ncu captures; "
                          "prints no result line)")
     ap.add_argument("--cpu-requests", type=int, default=64)
