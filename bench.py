@@ -331,7 +331,7 @@ def run_ours(args):
     # ---------------------------------------------------------------- prefill leg
     if not args.no_prefill:
         result["prefill"] = run_prefill(args, world, peaks, peak_src, flush)
-        result["gpu_launches"] += 2 * args.steps
+        result["gpu_launches"] += result["prefill"].pop("_launches")
 
     # ---------------------------------------------------------------- other workloads (optional)
     if args.extended:
@@ -417,13 +417,14 @@ def run_prefill(args, world, peaks, peak_src, flush):
     import torch
 
     from position_agnostic_paged_b200 import accounting
+    from position_agnostic_paged_b200 import lazy_attn as la
     from position_agnostic_paged_b200 import workloads as W
     from position_agnostic_paged_b200.runner import DevicePool, DeviceStep
 
     wl = W.make("prefill_8b")
     step = wl.steps[0]
     pool = DevicePool(wl).setup()
-    ds = DeviceStep(pool, step)
+    ds = DeviceStep(pool, step, with_plain=not args.no_compare)
     _prepare_step_writes(ds)
     flops = accounting.prefill_flops(step.visible_pairs, wl.hq, wl.d)
 
@@ -443,7 +444,35 @@ def run_prefill(args, world, peaks, peak_src, flush):
     all_flops = sum_over_ranks(world, float(flops))
     achieved = flops / (attn_avg * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    comparison = None
+    if not args.no_compare:
+        # the same chunk through the comparison paths: rotation off (keys materialised once,
+        # outside the timing), and materialise-then-attend (the materialisation timed too)
+        def plain_step(ev):
+            ds.attend_plain()
+
+        def mat_step(ev):
+            ds.materialize()
+            ds.attend_plain()
+
+        ds.materialize()
+        plain_total, _ = timed_steps(plain_step, args.steps, args.warmup, flush, world)
+        mat_total, _ = timed_steps(mat_step, args.steps, args.warmup, flush, world)
+        torch.cuda.synchronize()
+        comparison = {
+            "lazy_prefill_attn_ms": round(attn_avg, 5),
+            "plain_prefill_attn_ms": round(max_over_ranks(world, plain_total / args.steps), 5),
+            "materialize_then_attend_ms": round(max_over_ranks(world, mat_total / args.steps), 5),
+            "materialized_k_bytes": int(ds.k_mat.numel() * 2),
+            "max_abs_lazy_minus_plain": float((ds.out.float() - ds.out_plain.float()).abs().max().item()),
+        }
+    # attention launches per call: the prefill kernel, plus the combine kernel when the workspace
+    # lets the last wave's units run split
+    per_call = 2 if ds.workspace.numel() >= 16 and la.prefill_workspace_bytes(
+        ds.cfg, step.num_req, step.total_q, ds.max_q, ds.max_words) > 0 else 1
+    launches = (1 + per_call) * args.steps + ((per_call + 1 + per_call) * args.steps if comparison else 0)
     return {
+        "_launches": launches,
         "workload": "prefill_8b: Llama-3.1-8B shapes, 16 requests x 256 causal query tokens over 10 Zipf(1.0) "
                     "docs x 512 (5376 keys), 1000-doc pool",
         "value": round(all_flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
@@ -452,6 +481,7 @@ def run_prefill(args, world, peaks, peak_src, flush):
         "roofline": {"bound": "tensor", "kernel": "lazy_prefill_attn", "achieved": round(achieved, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_source": peak_src,
                      "traffic": traffic_for("prefill_8b", "prefill_tc.cu")},
+        **({"comparison": comparison} if comparison else {}),
     }
 
 

@@ -99,7 +99,8 @@ class DeviceCase:
         q_pos0 = []
         for r in range(n):
             qp = c.q_pos[c.cu_q[r]:c.cu_q[r + 1]]
-            assert np.array_equal(qp, qp[0] + np.arange(qp.size)), "prefill: contiguous query positions"
+            assert qp.size == 0 or np.array_equal(qp, qp[0] + np.arange(qp.size)), \
+                "prefill: contiguous query positions"
             q_pos0.append(int(qp[0]) if qp.size else 0)
         total_q = int(c.cu_q[-1])
         max_q = int(np.diff(c.cu_q).max())

@@ -201,6 +201,62 @@ def test_scattered_document_blocks(kind, scatter):
     assert dc.status() == 0
 
 
+# ----------------------------------------------------------------------------- limits of the format
+@pytest.mark.parametrize("kind", ["decode", "prefill"])
+def test_offsets_near_the_15_bit_limit(kind):
+    """Segment offsets up to 32767 (the largest the table word holds) with positions beyond it:
+    the rotation angles of keys and queries stay exact at those positions."""
+    segs = [(0, 32000, 700), (700, 32767, 40), (740, 5, 30)]
+    qp = [32820] if kind == "decode" else list(range(32800, 32830))
+    case = make_case(41, hq=32, hkv=8, d=128, requests=[(segs, qp)])
+    dc = DeviceCase(case)
+    ref = oracle.attend(**case.oracle_kwargs())
+    got = dc.decode() if kind == "decode" else dc.prefill()
+    check(got, ref, max_abs=edge_max_abs(case), what=f"{kind} offsets near 2^15")
+    assert dc.status() == 0
+
+
+@pytest.mark.parametrize("kind", ["decode", "prefill"])
+def test_block_ids_near_the_17_bit_limit(kind):
+    """A pool of 2^17 blocks (the largest the table word addresses) with the documents scattered
+    over it, so that most words carry block ids far above 2^16."""
+    segs = [(0, 0, 200), (300, 210, 130)]
+    qp = [400] if kind == "decode" else list(range(340, 400))
+    case = make_case(43, hq=16, hkv=1, d=128, requests=[(segs, qp)])
+    nb = (200 + 15) // 16 + (130 + 15) // 16
+    dc = DeviceCase(case, extra_blocks=(1 << 17) - nb, scatter_seed=11)
+    assert int(dc.phys[:nb].max()) > (1 << 16)
+    ref = oracle.attend(**case.oracle_kwargs())
+    got = dc.decode() if kind == "decode" else dc.prefill()
+    check(got, ref, max_abs=edge_max_abs(case), what=f"{kind} block ids near 2^17")
+    assert dc.status() == 0
+
+
+def test_request_with_an_empty_table_among_others():
+    """A request that attends to nothing (no table words) gives zero rows; its neighbours are
+    unaffected."""
+    reqs = [([(0, 0, 64)], [80]), ([], [10]), ([(64, 100, 33)], [140])]
+    case = make_case(47, hq=32, hkv=8, d=128, requests=reqs)
+    dc = DeviceCase(case)
+    ref = oracle.attend(**case.oracle_kwargs())
+    out = dc.decode()
+    assert np.array_equal(out[32:64], np.zeros((32, 128)))
+    check(out, ref, max_abs=edge_max_abs(case), what="decode with an empty table")
+    assert dc.status() == 0
+
+
+def test_prefill_request_with_no_query_tokens():
+    """A prefill chunk of zero tokens between two others: nothing is written for it and the
+    others are correct."""
+    reqs = [([(0, 0, 64)], list(range(64, 80))), ([(64, 0, 32)], []), ([(96, 10, 50)], list(range(60, 90)))]
+    case = make_case(53, hq=32, hkv=8, d=128, requests=reqs)
+    dc = DeviceCase(case)
+    ref = oracle.attend(**case.oracle_kwargs())
+    check(dc.prefill(), ref, max_abs=edge_max_abs(case), what="prefill with an empty chunk")
+    check(dc.prefill(split=False), ref, max_abs=edge_max_abs(case), what="prefill with an empty chunk, unsplit")
+    assert dc.status() == 0
+
+
 def test_queries_that_see_nothing_give_zero_rows():
     case = make_case(5, hq=8, hkv=2, d=128, requests=[([(0, 100, 20)], [50]), ([(20, 0, 16)], [15])])
     dc = DeviceCase(case)
