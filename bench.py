@@ -55,7 +55,7 @@ TRAFFIC = {
     #     -k regex:decode_split -s 3 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu --no-compare --no-e2e
     "decode_8b": {"sha": "1882d73735d88144", "bytes": 782188544 + 7172352},
     # the same with -k regex:prefill_tc
-    "prefill_8b": {"sha": "19cfa1b7f0e3a1be", "bytes": 302290432 + 27631616},
+    "prefill_8b": {"sha": "3eb263b89dd13961", "bytes": 305164032 + 27624704},
 }
 
 

@@ -73,6 +73,14 @@ typedef struct lazy_attn_cfg {
     int block_size;      /* must be 16 */
     float rope_base;     /* RoPE base, e.g. 500000; theta_i = base^(-2i/d) */
     float softmax_scale; /* <= 0 selects 1/sqrt(head_dim) */
+    /* Optional: head_dim/2 RoPE frequencies theta_i (radians per position), in
+     * place of base^(-2i/d) -- RoPE variants such as Llama-3.1 frequency
+     * scaling.  NULL selects base^(-2i/d).  Read during the call only (the
+     * caller keeps ownership); each value must be finite and >= 0, else
+     * LAZY_EINVAL.  The deferred rotation is unchanged: every angle is
+     * (position difference) x theta_i.  The pages name other relative
+     * encodings as within reach of the method but fix no table. */
+    const double *rope_theta;
 } lazy_attn_cfg;
 
 /* Host-side return codes. */

@@ -17,6 +17,7 @@ from .oracle import (  # noqa: F401
     unpack_word,
     pack_meta,
     rope,
+    llama31_theta,
     kv_write,
     expand_table,
     attend,

@@ -30,7 +30,9 @@
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   - RoPE uses the rotate-half pairing (component i with component i + d/2)
- *     and frequencies theta_i = base^(-2i/d); no frequency scaling.
+ *     and frequencies theta_i = base^(-2i/d) unless a frequency table is set
+ *     (RoPE variants such as Llama-3.1 frequency scaling, computed here by
+ *     oracle_llama31_theta from the published rule).
  *   - Softmax scale 1/sqrt(d) unless given; no soft-cap.
  *   - Causal rule: key at position t is visible to a query at position p iff
  *     t <= p.  A query that sees no key produces a zero row.
@@ -52,6 +54,10 @@
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
+#endif
+
+#ifndef M_PI
+#define M_PI 3.14159265358979323846
 #endif
 
 #define OR_OK 0
@@ -131,9 +137,51 @@ uint32_t oracle_pack_meta(int32_t block_index_in_segment, int32_t n_valid)
 /* RoPE ([CORE]: positional encoding applied to keys and queries).           */
 /* ------------------------------------------------------------------------- */
 
+/* Optional frequency table: when set for d/2 components, theta_i = table[i].
+ * Set before a call and cleared after it by the Python wrapper (one call at a
+ * time; OpenMP threads only read it). */
+static double g_theta[512];
+static int g_theta_n = 0;
+
+void oracle_set_rope_theta(const double *theta, int half)
+{
+    if (!theta || half <= 0 || half > 512) {
+        g_theta_n = 0;
+        return;
+    }
+    memcpy(g_theta, theta, sizeof(double) * (size_t)half);
+    g_theta_n = half;
+}
+
 static double rope_theta(int i, int d, double base)
 {
+    if (g_theta_n == d / 2) return g_theta[i];
     return pow(base, -2.0 * (double)i / (double)d);
+}
+
+/* Llama-3.1 frequency scaling of the RoPE frequencies (the "llama3" rope type
+ * of the Llama 3.1 model configuration): with f_i = base^(-2i/d) and its
+ * wavelength 2*pi/f_i, components whose wavelength is below
+ * original_max/high_factor keep f_i, those above original_max/low_factor get
+ * f_i/factor, and in between f_i is interpolated linearly in the ratio
+ * original_max/wavelength, from f_i/factor at low_factor to f_i at
+ * high_factor. */
+void oracle_llama31_theta(double base, int d, double factor, double low_factor, double high_factor,
+                          double original_max, double *theta)
+{
+    const double lo_wl = original_max / low_factor, hi_wl = original_max / high_factor;
+    for (int i = 0; i < d / 2; ++i) {
+        const double f = pow(base, -(2.0 * i) / d);   /* the unscaled frequency */
+        const double wl = 2.0 * M_PI / f;
+        if (wl < hi_wl) {
+            theta[i] = f;
+        } else if (wl > lo_wl) {
+            theta[i] = f / factor;
+        } else {
+            const double s = (original_max / wl - low_factor) / (high_factor - low_factor);
+            theta[i] = (1.0 - s) * f / factor + s * f;
+        }
+    }
 }
 
 /* y = RoPE(x, pos): for each pair (i, i + d/2) rotate by angle pos*theta_i. */

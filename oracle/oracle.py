@@ -88,6 +88,11 @@ def _bind(lib) -> None:
     lib.oracle_rope_rows_bf16.restype = ctypes.c_int
     lib.oracle_rope_rows_bf16.argtypes = [
         ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_double, _u16p, _i32p, _u16p]
+    lib.oracle_set_rope_theta.restype = None
+    lib.oracle_set_rope_theta.argtypes = [_f64p, ctypes.c_int]
+    lib.oracle_llama31_theta.restype = None
+    lib.oracle_llama31_theta.argtypes = [ctypes.c_double, ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                         ctypes.c_double, ctypes.c_double, _f64p]
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_set_num_threads.restype = None
@@ -96,6 +101,33 @@ def _bind(lib) -> None:
 
 def _p(a: np.ndarray, ct):
     return a.ctypes.data_as(ct)
+
+
+class _Theta:
+    """Sets the oracle's RoPE frequency table for one call (None: base^(-2i/d))."""
+
+    def __init__(self, lib, theta):
+        self.lib = lib
+        self.theta = None if theta is None else _c(theta, np.float64)
+
+    def __enter__(self):
+        if self.theta is not None:
+            self.lib.oracle_set_rope_theta(_p(self.theta, _f64p), int(self.theta.size))
+        return self
+
+    def __exit__(self, *exc):
+        if self.theta is not None:
+            self.lib.oracle_set_rope_theta(ctypes.cast(None, _f64p), 0)
+        return False
+
+
+def llama31_theta(base: float = 500000.0, d: int = 128, factor: float = 8.0, low_factor: float = 1.0,
+                  high_factor: float = 4.0, original_max: float = 8192.0) -> np.ndarray:
+    """RoPE frequencies with Llama-3.1 frequency scaling (the oracle's own computation)."""
+    out = np.empty(d // 2, np.float64)
+    _load().oracle_llama31_theta(float(base), int(d), float(factor), float(low_factor), float(high_factor),
+                                 float(original_max), _p(out, _f64p))
+    return out
 
 
 def _c(a, dtype) -> np.ndarray:
@@ -141,14 +173,16 @@ def pack_meta(block_index_in_segment: int, n_valid: int) -> int:
     return int(_load().oracle_pack_meta(int(block_index_in_segment), int(n_valid)))
 
 
-def rope(x, pos: int, base: float) -> np.ndarray:
+def rope(x, pos: int, base: float, theta=None) -> np.ndarray:
     x = _c(x, np.float64)
     y = np.empty_like(x)
-    _load().oracle_rope(_p(x, _f64p), int(x.shape[-1]), float(base), int(pos), _p(y, _f64p))
+    lib = _load()
+    with _Theta(lib, theta):
+        lib.oracle_rope(_p(x, _f64p), int(x.shape[-1]), float(base), int(pos), _p(y, _f64p))
     return y
 
 
-def kv_write(k_raw, v_raw, slot, local_j, k_pool, v_pool, blk_meta, base: float) -> int:
+def kv_write(k_raw, v_raw, slot, local_j, k_pool, v_pool, blk_meta, base: float, theta=None) -> int:
     """Applies the expected effect of a pool write in place on numpy arrays.
 
     k_raw, v_raw: uint16 [n_tok, Hkv, d]; k_pool, v_pool: uint16 [nb, Hkv, 16, d];
@@ -161,10 +195,12 @@ def kv_write(k_raw, v_raw, slot, local_j, k_pool, v_pool, blk_meta, base: float)
     assert k_pool.flags.c_contiguous and v_pool.flags.c_contiguous and blk_meta.flags.c_contiguous
     assert k_pool.dtype == np.uint16 and v_pool.dtype == np.uint16 and blk_meta.dtype == np.uint32
     n_tok, hkv, d = k_raw.shape
-    return int(_load().oracle_kv_write(
-        int(n_tok), int(hkv), int(d), float(base), _p(k_raw, _u16p), _p(v_raw, _u16p),
-        _p(slot, _i32p), _p(local_j, _i32p), int(k_pool.shape[0]),
-        _p(k_pool, _u16p), _p(v_pool, _u16p), _p(blk_meta, _u32p)))
+    lib = _load()
+    with _Theta(lib, theta):
+        return int(lib.oracle_kv_write(
+            int(n_tok), int(hkv), int(d), float(base), _p(k_raw, _u16p), _p(v_raw, _u16p),
+            _p(slot, _i32p), _p(local_j, _i32p), int(k_pool.shape[0]),
+            _p(k_pool, _u16p), _p(v_pool, _u16p), _p(blk_meta, _u32p)))
 
 
 def expand_table(words, blk_meta, num_blocks: int):
@@ -182,7 +218,7 @@ def expand_table(words, blk_meta, num_blocks: int):
 
 def attend(*, num_q_heads: int, num_kv_heads: int, rope_base: float, q_raw, cu_q, q_pos,
            seg_indptr, seg_src, seg_off, seg_len, k_tok, v_tok, sel_q=None, sel_h=None,
-           softmax_scale: float = 0.0, want_scores: bool = False, lib=None):
+           softmax_scale: float = 0.0, want_scores: bool = False, lib=None, rope_theta=None):
     """Materialised causal GQA attention in fp64.
 
     q_raw: uint16 [total_q, Hq, d]; k_tok, v_tok: uint16 [n_store, Hkv, d].
@@ -220,12 +256,14 @@ def attend(*, num_q_heads: int, num_kv_heads: int, rope_base: float, q_raw, cu_q
         ld = 0
         scores = None
         sp = ctypes.cast(None, _f64p)
-    rc = (lib or _load()).oracle_attend(
-        int(num_req), int(num_q_heads), int(num_kv_heads), int(d), float(rope_base),
-        float(softmax_scale), _p(q_raw, _u16p), _p(cu_q, _i32p), _p(q_pos, _i32p),
-        _p(seg_indptr, _i32p), _p(seg_src, _i32p), _p(seg_off, _i32p), _p(seg_len, _i32p),
-        _p(k_tok, _u16p), _p(v_tok, _u16p), int(n_sel), _p(sq, _i32p), _p(sh, _i32p),
-        _p(out, _f64p), sp, int(ld))
+    lib = lib or _load()
+    with _Theta(lib, rope_theta):
+        rc = lib.oracle_attend(
+            int(num_req), int(num_q_heads), int(num_kv_heads), int(d), float(rope_base),
+            float(softmax_scale), _p(q_raw, _u16p), _p(cu_q, _i32p), _p(q_pos, _i32p),
+            _p(seg_indptr, _i32p), _p(seg_src, _i32p), _p(seg_off, _i32p), _p(seg_len, _i32p),
+            _p(k_tok, _u16p), _p(v_tok, _u16p), int(n_sel), _p(sq, _i32p), _p(sh, _i32p),
+            _p(out, _f64p), sp, int(ld))
     if rc != 0:
         raise RuntimeError(f"oracle_attend failed with status {rc}")
     out = out[:n_rows]
@@ -234,13 +272,15 @@ def attend(*, num_q_heads: int, num_kv_heads: int, rope_base: float, q_raw, cu_q
     return out
 
 
-def rope_rows_bf16(k_raw, pos, base: float) -> np.ndarray:
+def rope_rows_bf16(k_raw, pos, base: float, theta=None) -> np.ndarray:
     """bf16(RoPE(k_raw[n], pos[n])) for uint16 k_raw [n, Hkv, d]."""
     k_raw = _c(k_raw, np.uint16)
     pos = _c(pos, np.int32)
     out = np.empty_like(k_raw)
     n, hkv, d = k_raw.shape
-    rc = _load().oracle_rope_rows_bf16(int(n), int(hkv), int(d), float(base), _p(k_raw, _u16p),
+    lib = _load()
+    with _Theta(lib, theta):
+        rc = lib.oracle_rope_rows_bf16(int(n), int(hkv), int(d), float(base), _p(k_raw, _u16p),
                                        _p(pos, _i32p), _p(out, _u16p))
     if rc != 0:
         raise RuntimeError(f"oracle_rope_rows_bf16 failed with status {rc}")

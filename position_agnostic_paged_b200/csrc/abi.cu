@@ -18,7 +18,7 @@ using namespace lazy;
 
 namespace {
 
-constexpr int kVersion = 100;
+constexpr int kVersion = 101;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -82,12 +82,17 @@ int check_cfg(const lazy_attn_cfg *cfg) {
     if (cfg->num_q_heads / cfg->num_kv_heads > 32) return LAZY_ESHAPE;
     if (cfg->num_kv_heads > 64) return LAZY_ESHAPE;
     if (!(cfg->rope_base > 1.0f) || !std::isfinite(cfg->rope_base)) return LAZY_EINVAL;
+    if (cfg->rope_theta)
+        for (int i = 0; i < 64; ++i)
+            if (!std::isfinite(cfg->rope_theta[i]) || cfg->rope_theta[i] < 0.0) return LAZY_EINVAL;
     return LAZY_OK;
 }
 
-void fill_rope(RopeTableHost &t, float base) {
-    // theta_i = base^(-2i/d) for the rotate-half pairs (i, i + d/2)
-    for (int i = 0; i < 64; ++i) t.theta[i] = std::pow(static_cast<double>(base), -2.0 * i / 128.0);
+void fill_rope(RopeTableHost &t, const lazy_attn_cfg *cfg) {
+    // theta_i for the rotate-half pairs (i, i + d/2): the caller's table, else base^(-2i/d)
+    for (int i = 0; i < 64; ++i)
+        t.theta[i] = cfg->rope_theta ? cfg->rope_theta[i]
+                                     : std::pow(static_cast<double>(cfg->rope_base), -2.0 * i / 128.0);
 }
 
 float scale_log2(const lazy_attn_cfg *cfg) {
@@ -126,7 +131,7 @@ int attn_common(const lazy_attn_cfg *cfg, AttnParams &p, int num_req, const uint
     p.num_blocks = num_blocks;
     p.max_words = max_words;
     p.scale_log2 = scale_log2(cfg);
-    fill_rope(p.rope, cfg->rope_base);
+    fill_rope(p.rope, cfg);
     return LAZY_OK;
 }
 
@@ -258,7 +263,7 @@ int lazy_kv_write(const lazy_attn_cfg *cfg, const uint16_t *k_raw, const uint16_
     p.hkv = cfg->num_kv_heads;
     p.num_blocks = num_blocks;
     p.d_status = d_status;
-    fill_rope(p.rope, cfg->rope_base);
+    fill_rope(p.rope, cfg);
     return launch_rc(launch_kv_write(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -313,7 +318,7 @@ int lazy_materialize_k(const lazy_attn_cfg *cfg, const uint32_t *table, int tota
     p.hkv = cfg->num_kv_heads;
     p.num_blocks = num_blocks;
     p.d_status = d_status;
-    fill_rope(p.rope, cfg->rope_base);
+    fill_rope(p.rope, cfg);
     return launch_rc(launch_materialize(p, static_cast<cudaStream_t>(stream)));
 }
 

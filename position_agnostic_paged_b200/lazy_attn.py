@@ -37,21 +37,30 @@ class LazyAttnError(RuntimeError):
 
 class LazyAttnCfg(ctypes.Structure):
     _fields_ = [("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
-                ("block_size", ctypes.c_int), ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float)]
+                ("block_size", ctypes.c_int), ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+                ("rope_theta", ctypes.POINTER(ctypes.c_double))]
 
 
 @dataclass(frozen=True)
 class Cfg:
+    """rope_theta: optional head_dim/2 RoPE frequencies (e.g. rope.llama31_theta()) in place of
+    rope_base^(-2i/head_dim)."""
     num_q_heads: int
     num_kv_heads: int
     rope_base: float = 500000.0
     head_dim: int = 128
     block_size: int = 16
     softmax_scale: float = 0.0
+    rope_theta: tuple | None = None
 
     def c(self) -> LazyAttnCfg:
-        return LazyAttnCfg(self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
-                           float(self.rope_base), float(self.softmax_scale))
+        st = LazyAttnCfg(self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
+                         float(self.rope_base), float(self.softmax_scale), None)
+        if self.rope_theta is not None:
+            arr = (ctypes.c_double * len(self.rope_theta))(*[float(x) for x in self.rope_theta])
+            st._theta_keepalive = arr
+            st.rope_theta = ctypes.cast(arr, ctypes.POINTER(ctypes.c_double))
+        return st
 
 
 _vp, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t

@@ -25,9 +25,11 @@ def _i32(a, dev):
 
 
 class DeviceCase:
-    def __init__(self, case, dev="cuda", extra_blocks: int = 0, scatter_seed: int | None = None):
+    def __init__(self, case, dev="cuda", extra_blocks: int = 0, scatter_seed: int | None = None,
+                 rope_theta=None):
         self.case = case
-        self.cfg = la.Cfg(case.hq, case.hkv, rope_base=case.base)
+        self.cfg = la.Cfg(case.hq, case.hkv, rope_base=case.base,
+                          rope_theta=None if rope_theta is None else tuple(float(x) for x in rope_theta))
         docs = {}
         for g in range(case.seg_src.size):
             src, ln = int(case.seg_src[g]), int(case.seg_len[g])

@@ -31,7 +31,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_strerror():
-    assert la.version() == 100
+    assert la.version() == 101
     for code in (0, -1, -2, -3, -4, -5):
         assert la.strerror(code) and la.strerror(code) != "unknown error"
 

@@ -257,6 +257,84 @@ def test_prefill_request_with_no_query_tokens():
     assert dc.status() == 0
 
 
+# ----------------------------------------------------------------------------- RoPE frequency tables
+def _llama31_tables():
+    """The product's and the oracle's Llama-3.1 frequency tables: two independent computations of
+    the published rule, which must agree."""
+    from position_agnostic_paged_b200 import rope as prope
+    tp = np.array(prope.llama31_theta())
+    to = oracle.llama31_theta()
+    np.testing.assert_allclose(tp, to, rtol=1e-14)
+    return tp, to
+
+
+@pytest.mark.parametrize("kind", ["decode", "prefill"])
+def test_llama31_frequency_table(kind):
+    """Attention with Llama-3.1-scaled RoPE frequencies passed through the configuration, at
+    positions near 32k where the scaling changes the result."""
+    tp, to = _llama31_tables()
+    segs = [(0, 30000, 300), (300, 31000, 200), (500, 100, 64)]
+    qp = [31300] if kind == "decode" else list(range(31250, 31290))
+    case = make_case(61, hq=32, hkv=8, d=128, requests=[(segs, qp)])
+    dc = DeviceCase(case, rope_theta=tp)
+    ref = oracle.attend(**case.oracle_kwargs(), rope_theta=to)
+    tol = edge_max_abs(case)
+    assert np.abs(ref - oracle.attend(**case.oracle_kwargs())).max() > 3 * tol   # the table matters here
+    got = dc.decode() if kind == "decode" else dc.prefill()
+    check(got, ref, max_abs=tol, what=f"{kind} llama-3.1 frequencies, lazy")
+    got_p = dc.decode(plain=True) if kind == "decode" else dc.prefill(plain=True)
+    check(got_p, ref, max_abs=tol, what=f"{kind} llama-3.1 frequencies, plain")
+    assert dc.status() == 0
+
+
+def test_kv_write_with_a_frequency_table():
+    tp, to = _llama31_tables()
+    rng = np.random.default_rng(71)
+    hkv, d, nb = 4, 128, 40
+    n = 400
+    k = (rng.standard_normal((n, hkv, d)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    v = (rng.standard_normal((n, hkv, d)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    slot = rng.permutation(nb * 16)[:n].astype(np.int32)
+    # a token's slot inside its block is its local index mod 16
+    local_j = (16 * rng.integers(0, 1875, n) + slot % 16).astype(np.int32)
+    cfg = la.Cfg(hkv * 2, hkv, rope_theta=tuple(tp))
+    dev = "cuda"
+    kp = torch.zeros((nb, hkv, 16, d), dtype=torch.bfloat16, device=dev)
+    vp = torch.zeros_like(kp)
+    meta = torch.zeros(nb, dtype=torch.int32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    u16 = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    la.kv_write(cfg, u16(k), u16(v), torch.from_numpy(slot).to(dev), torch.from_numpy(local_j).to(dev),
+                kp, vp, meta, st)
+    okp = np.zeros((nb, hkv, 16, d), np.uint16)
+    ovp = okp.copy()
+    ometa = np.zeros(nb, np.uint32)
+    assert oracle.kv_write(k, v, slot, local_j, okp, ovp, ometa, 500000.0, theta=to) == 0
+    gk = kp.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(vp.view(torch.int16).cpu().numpy().view(np.uint16), ovp)
+    assert np.array_equal(meta.cpu().numpy().view(np.uint32), ometa)
+    # The kernel rotates in fp32 (angle reduced in fp64, sincosf) and rounds once to bf16; the
+    # oracle works in fp64.  Where a*c - b*s nearly cancels, the fp32 error (about 2^-24 of the
+    # inputs' magnitude) can exceed one bf16 ulp of the small result, so the bound is one ulp of
+    # the result plus 2^-20 absolute (inputs are N(0,1), |a|, |b| < 8), and multi-ulp cases must
+    # be rare.
+    g, o = bits_to_f64(gk), bits_to_f64(okp)
+    diff = np.abs(gk.astype(np.int32) - okp.astype(np.int32))
+    err = np.abs(g - o)
+    ok = err <= np.abs(o) * 2.0 ** -7 + 2.0 ** -20
+    if not ok.all():
+        idx = np.argwhere(~ok)[:6]
+        rows = []
+        for b_, h_, s_, i_ in idx:
+            tok = np.where(slot == b_ * 16 + s_)[0]
+            jj = int(local_j[tok[0]]) if tok.size else -1
+            rows.append(f"blk {b_} head {h_} slot {s_} comp {i_} j {jj}: gpu {g[b_, h_, s_, i_]:.6g} "
+                        f"oracle {o[b_, h_, s_, i_]:.6g} ulps {diff[b_, h_, s_, i_]}")
+        raise AssertionError(f"{(~ok).sum()} keys outside the bound; max ulps {diff.max()}\n" + "\n".join(rows))
+    assert (diff > 1).mean() < 1e-4 and (diff != 0).mean() < 0.02
+    assert int(st.item()) == 0
+
+
 def test_queries_that_see_nothing_give_zero_rows():
     case = make_case(5, hq=8, hkv=2, d=128, requests=[([(0, 100, 20)], [50]), ([(20, 0, 16)], [15])])
     dc = DeviceCase(case)

@@ -283,3 +283,46 @@ def test_rope_rows_bf16_matches_rotation():
     assert np.array_equal(out[0], k[0])
     exact = _rope_complex(bits_to_f64(k), pos.astype(np.float64), BASE)
     assert (np.abs(bits_to_f64(out) - exact) <= np.abs(exact) * 2.0 ** -8 + 1e-30).all()
+
+
+# ----------------------------------------------------------------------------- RoPE frequency tables
+def test_llama31_table_regions_by_hand():
+    """base 5e5, d 128, factor 8, low/high factors 1/4, original context 8192.  A component keeps its
+    frequency when its wavelength 2*pi*5e5^(i/64) is below 8192/4 = 2048, i.e. 5e5^(i/64) < 325.95,
+    i < 64*ln(325.95)/ln(5e5) = 28.22 -> i = 0..28; it is divided by 8 when the wavelength exceeds
+    8192, i.e. i > 64*ln(1303.8)/ln(5e5) = 34.99 -> i = 35..63; i = 29..34 are interpolated."""
+    th = oracle.llama31_theta(500000.0, 128, 8.0, 1.0, 4.0, 8192.0)
+    plain = np.array([500000.0 ** (-i / 64.0) for i in range(64)])
+    assert np.array_equal(th[:29], plain[:29])
+    np.testing.assert_allclose(th[35:], plain[35:] / 8.0, rtol=0, atol=0)
+    mid = th[29:35] / plain[29:35]
+    assert np.all(mid < 1.0) and np.all(mid > 1.0 / 8.0)
+    assert np.all(np.diff(th) < 0)                      # frequencies still decrease with i
+
+
+def test_llama31_table_factor_one_and_continuity():
+    plain = oracle.llama31_theta(10000.0, 64, 1.0, 1.0, 4.0, 2048.0)
+    np.testing.assert_allclose(plain, [10000.0 ** (-2.0 * i / 64) for i in range(32)], rtol=1e-15)
+    # a frequency sitting exactly on either boundary gets the same value from both sides
+    import math
+    base, d, orig = 500000.0, 128, 8192.0
+    for wl_edge, expect_ratio in ((orig / 4.0, 1.0), (orig / 1.0, 1.0 / 8.0)):
+        # choose base so that component 1 has exactly that wavelength
+        f = 2 * math.pi / wl_edge
+        b = f ** (-d / 2.0)
+        th = oracle.llama31_theta(b, d, 8.0, 1.0, 4.0, orig)
+        assert abs(th[1] / f - expect_ratio) < 1e-12
+
+
+def test_rope_with_a_table_is_relative_and_default_table_matches():
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal(128)
+    k = rng.standard_normal(128)
+    th = oracle.llama31_theta()
+    s1 = oracle.rope(q, 9000, 500000.0, theta=th) @ oracle.rope(k, 1234, 500000.0, theta=th)
+    s2 = oracle.rope(q, 9000 + 77777, 500000.0, theta=th) @ oracle.rope(k, 1234 + 77777, 500000.0, theta=th)
+    assert abs(s1 - s2) < 1e-9 * max(1.0, abs(s1))
+    dflt = np.array([500000.0 ** (-2.0 * i / 128) for i in range(64)])
+    np.testing.assert_array_equal(oracle.rope(q, 4321, 500000.0, theta=dflt), oracle.rope(q, 4321, 500000.0))
+    # and the scaled table really changes long-wavelength components
+    assert not np.allclose(oracle.rope(q, 4321, 500000.0, theta=th), oracle.rope(q, 4321, 500000.0))
