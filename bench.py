@@ -623,6 +623,18 @@ def run_profile_case(args):
     log(f"[profile-case] {args.profile_case}: {args.steps} launches, status {pool.status()}")
 
 
+def run_cache_sim(args):
+    """Cache-hit ratios of position-agnostic caching against position-aware (re-encoding and
+    exact-offset) and prefix caching, at a 1 GB KV budget of Llama-3.1-8B geometry, for three Zipf
+    exponents of document popularity; host only, one JSON line per exponent."""
+    from position_agnostic_paged_b200 import cache_sim
+    t0 = time.perf_counter()
+    for row in cache_sim.compare(n_requests=args.cache_requests):
+        print(json.dumps({"metric": "cache_hit_ratio", "unit": "fraction of document blocks",
+                          "data": "synthetic", "requests": args.cache_requests, **row}), flush=True)
+    log(f"[cache-sim] {time.perf_counter() - t0:.1f} s")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -639,12 +651,18 @@ def main():
     ap.add_argument("--profile-case", choices=["prefill_small", "decode_small", "decode_mqa_small"],
                     help="launch only the attention kernel of a small case --steps times (for ncu captures; "
                          "prints no result line)")
+    ap.add_argument("--cache-sim", action="store_true",
+                    help="host-side cache-hit simulation of the caching policies (no GPU; prints one line "
+                         "per Zipf exponent)")
+    ap.add_argument("--cache-requests", type=int, default=20000)
     ap.add_argument("--cpu-requests", type=int, default=64)
     ap.add_argument("--ref-requests", type=int, default=2)
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.profile_case:
+    if args.cache_sim:
+        run_cache_sim(args)
+    elif args.profile_case:
         run_profile_case(args)
     elif args.impl == "reference":
         run_reference(args)

@@ -11,6 +11,8 @@
  *         Technical Summary: Core Concept: Deferred Positional Encoding;
  *         Technical Implementation: Prefilling; Technical Implementation:
  *         Decoding; Mathematical Equivalence; Key Contributions.
+ *   [RES] gist.science, same title -- Experimental Results (cache hit
+ *         ratios under a KV budget).
  *
  * Conventions for every entry point
  *   - Pointers are DEVICE pointers unless marked "host".  bf16 tensors are
@@ -200,8 +202,9 @@ int lazy_prefill_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int
 
 /* ---- comparison paths (the position-aware alternative the pages argue against) ---- */
 
-/* Materialises position-adjusted keys ([ABS]: "memory materialization for
- * positional re-encoding"): for every table word w (global index into table,
+/* Materialises position-adjusted keys ([ABS]: copying keys re-encoded for
+ * their positions is the cost the method avoids): for every table word w
+ * (global index into table,
  * 0 <= w < total_words) with block b and offset o,
  *   k_mat[w][h][s][:] = bf16_rne(RoPE(k_pool[b][h][s][:], o))   for s < n_valid(b)
  *   k_mat[w][h][s][:] = 0                                        otherwise
@@ -229,6 +232,37 @@ int lazy_plain_prefill_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, con
                             const uint32_t *blk_meta, const uint16_t *k_mat, int total_words,
                             const uint16_t *v_pool, int num_blocks, uint16_t *out, void *workspace,
                             size_t ws_bytes, int *d_status, void *stream);
+
+/* ---- block cache (host side): what the shared pool holds ---- */
+
+/* A keyed LRU cache over pool blocks 0 .. capacity_blocks-1 ([ABS], [RES]:
+ * one physical copy per document, reused at any position; the pages compare
+ * its hit ratio with position-aware caching, one copy per (document, offset),
+ * and with prefix caching).  The caching policy is the caller's key: the
+ * document id (position-agnostic), a hash of (document, offset)
+ * (position-aware) or of the whole preceding document sequence (prefix).
+ * Host memory only; not thread-safe (one cache per scheduling thread).
+ * Returns NULL for capacity_blocks <= 0, > LAZY_MAX_BLOCKS or no memory. */
+typedef struct lazy_block_cache lazy_block_cache;
+lazy_block_cache *lazy_cache_create(int64_t capacity_blocks);
+void lazy_cache_destroy(lazy_block_cache *cache);
+
+/* One use of the entry `key` of n_blocks blocks.  Hit: writes its block ids
+ * to blocks[0..n_blocks-1], makes it the most recently used entry, returns 1
+ * (LAZY_EINVAL if it was cached with another size).  Miss: evicts least
+ * recently used entries until n_blocks are free, allocates them (consecutive
+ * when one free extent holds them all), writes their ids and returns 0; the
+ * caller then writes the document's keys and values there (lazy_kv_write).
+ * An entry larger than the whole cache is counted as a miss and not cached:
+ * LAZY_ERANGE. */
+int lazy_cache_access(lazy_block_cache *cache, uint64_t key, int32_t n_blocks, int32_t *blocks);
+
+/* 1 if key is cached, 0 if not. */
+int lazy_cache_contains(const lazy_block_cache *cache, uint64_t key);
+
+/* stats[8]: hits, misses, hit blocks, miss blocks, evictions, blocks in use,
+ * cached entries, free extents. */
+int lazy_cache_stats(const lazy_block_cache *cache, int64_t *stats);
 
 /* ---- test export ---- */
 

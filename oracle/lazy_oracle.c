@@ -416,8 +416,9 @@ void oracle_set_num_threads(int n)
 }
 
 /* Keys rotated eagerly at given logical positions and rounded to bf16: the
- * content a position-aware cache would hold ([ABS]: "memory materialization
- * for positional re-encoding").  Used to check a materialised-key copy.
+ * content a position-aware cache would hold ([ABS]: a copy re-encoded for its
+ * positions, the cost the method avoids).  Used to check a materialised-key
+ * copy.
  *   out[n][h][:] = bf16(RoPE(k_raw[n][h][:], pos[n])) */
 int oracle_rope_rows_bf16(int64_t n, int num_kv_heads, int head_dim, double rope_base,
                           const uint16_t *k_raw, const int32_t *pos, uint16_t *out)

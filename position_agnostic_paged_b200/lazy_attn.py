@@ -26,6 +26,7 @@ EXPORTED = [
     "lazy_prefill_workspace_bytes", "lazy_prefill_attn",
     "lazy_materialize_k", "lazy_plain_decode_attn", "lazy_plain_prefill_attn",
     "lazy_debug_decode_table", "lazy_decode_attn_noalloc", "lazy_decode_noalloc_capacity",
+    "lazy_cache_create", "lazy_cache_destroy", "lazy_cache_access", "lazy_cache_contains", "lazy_cache_stats",
 ]
 
 
@@ -90,6 +91,11 @@ def _load():
         "lazy_debug_decode_table": (_i, [_vp, _i64, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
         "lazy_decode_attn_noalloc": (_i, [_cfgp, _vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
         "lazy_decode_noalloc_capacity": (_sz, []),
+        "lazy_cache_create": (_vp, [_i64]),
+        "lazy_cache_destroy": (None, [_vp]),
+        "lazy_cache_access": (_i, [_vp, ctypes.c_uint64, ctypes.c_int32, _vp]),
+        "lazy_cache_contains": (_i, [_vp, ctypes.c_uint64]),
+        "lazy_cache_stats": (_i, [_vp, _vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -229,3 +235,49 @@ def decode_attn_noalloc(cfg: Cfg, q_raw, q_pos, table, table_indptr, max_words: 
         ctypes.byref(c), _ptr(q_raw), _ptr(q_pos), int(q_pos.numel()), _ptr(table), _ptr(table_indptr),
         int(max_words), _ptr(blk_meta), _ptr(k_pool), _ptr(v_pool), int(k_pool.shape[0]), _ptr(out),
         _ptr(d_status), _stream(stream)))
+
+
+class BlockCache:
+    """Host-side LRU cache of pool blocks (lazy_cache_*): key -> the blocks of one cached entry.
+
+    access(key, n_blocks) returns (hit, block_ids); on a miss the blocks are freshly allocated
+    (after evicting least recently used entries) and the caller writes the entry there.  An entry
+    larger than the cache is counted as a miss and returns (False, None).
+    """
+
+    STAT_NAMES = ("hits", "misses", "hit_blocks", "miss_blocks", "evictions", "used_blocks", "entries",
+                  "free_extents")
+
+    def __init__(self, capacity_blocks: int):
+        self._h = _lib.lazy_cache_create(int(capacity_blocks))
+        if not self._h:
+            raise LazyAttnError("lazy_cache_create", LAZY_EINVAL)
+        self.capacity = int(capacity_blocks)
+        self._buf = (ctypes.c_int32 * 1)()
+
+    def close(self) -> None:
+        if self._h:
+            _lib.lazy_cache_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    def access(self, key: int, n_blocks: int):
+        if len(self._buf) < n_blocks:
+            self._buf = (ctypes.c_int32 * max(n_blocks, 2 * len(self._buf)))()
+        rc = _lib.lazy_cache_access(self._h, ctypes.c_uint64(int(key) & 0xFFFFFFFFFFFFFFFF), int(n_blocks),
+                                    ctypes.cast(self._buf, ctypes.c_void_p))
+        if rc == LAZY_ERANGE:
+            return False, None
+        if rc < 0:
+            raise LazyAttnError("lazy_cache_access", rc)
+        return rc == 1, np.frombuffer(self._buf, dtype=np.int32, count=n_blocks).copy()
+
+    def contains(self, key: int) -> bool:
+        return _lib.lazy_cache_contains(self._h, ctypes.c_uint64(int(key) & 0xFFFFFFFFFFFFFFFF)) == 1
+
+    def stats(self) -> dict:
+        out = (ctypes.c_int64 * 8)()
+        _check("lazy_cache_stats", _lib.lazy_cache_stats(self._h, ctypes.cast(out, ctypes.c_void_p)))
+        return dict(zip(self.STAT_NAMES, [int(x) for x in out]))

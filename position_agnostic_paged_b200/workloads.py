@@ -383,3 +383,21 @@ def make(name: str, seed: int | None = None, **overrides) -> Workload:
 
 def with_overrides(step: Step, **kw) -> Step:
     return dataclasses.replace(step, **kw)
+
+
+# ----------------------------------------------------------------------------- cache-hit streams
+def cache_stream(seed: int, n_docs: int = 4000, doc_len=(128, 2048), docs_per_req: int = 8,
+                 alpha: float = 1.0, n_requests: int = 20000):
+    """A seeded stream of RAG requests for cache simulations: per request, docs_per_req distinct
+    documents drawn from a finite Zipf(alpha) popularity (rank k has weight k^-alpha), in random
+    order.  Returns (doc_tokens [n_docs] int64, requests [n_requests][docs_per_req] int64)."""
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(doc_len[0], doc_len[1] + 1, n_docs).astype(np.int64)
+    pop = rng.permutation(n_docs)             # document id of popularity rank k
+    w = zipf_probs(n_docs, alpha)
+    reqs = np.empty((n_requests, docs_per_req), np.int64)
+    for r in range(n_requests):
+        ranks = rng.choice(n_docs, size=docs_per_req, replace=False, p=w)
+        reqs[r] = pop[ranks]
+        rng.shuffle(reqs[r])
+    return lens, reqs

@@ -17,7 +17,8 @@ HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "la
 def _declared():
     txt = open(HEADER).read()
     txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
-    names = re.findall(r"^\s*(?:const\s+)?(?:int|size_t|char\s*\*|void)\s*\*?\s*(lazy_\w+)\s*\(", txt, flags=re.M)
+    names = re.findall(r"^\s*(?:const\s+)?(?:int|size_t|char\s*\*|void|lazy_block_cache)\s*\*?\s*(lazy_\w+)\s*\(",
+                       txt, flags=re.M)
     return sorted(set(names))
 
 
