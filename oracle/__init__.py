@@ -18,6 +18,7 @@ from .oracle import (  # noqa: F401
     pack_meta,
     rope,
     llama31_theta,
+    alibi_slopes,
     kv_write,
     expand_table,
     attend,

@@ -44,6 +44,13 @@
  *     index of the block's first token inside its segment and n_valid (1..16)
  *     the number of written slots.
  *   - bf16 values round to nearest, ties to even.
+ *   - ALiBi ([CON] names it among the relative encodings the method extends
+ *     to): when per-head slopes m_h are set, nothing is rotated and the score
+ *     of query head h at position p for the key at position t gets the linear
+ *     penalty -m_h * (p - t), with the distance p - t = p - o - j taken from
+ *     the same logical positions the RoPE path uses (Press, Smith and Lewis,
+ *     "Train Short, Test Long: Attention with Linear Biases", 2022, for the
+ *     bias and for the default slopes, oracle_alibi_slopes).
  *
  * Every function is plain C99; OpenMP (if enabled) only splits independent
  * output rows across threads.
@@ -151,6 +158,38 @@ void oracle_set_rope_theta(const double *theta, int half)
     }
     memcpy(g_theta, theta, sizeof(double) * (size_t)half);
     g_theta_n = half;
+}
+
+/* Optional ALiBi slopes, one per query head; set and cleared around a call
+ * like the frequency table.  While set, oracle_attend rotates nothing. */
+static double g_alibi[4096];
+static int g_alibi_n = 0;
+
+void oracle_set_alibi(const double *slopes, int n)
+{
+    if (!slopes || n <= 0 || n > 4096) {
+        g_alibi_n = 0;
+        return;
+    }
+    memcpy(g_alibi, slopes, sizeof(double) * (size_t)n);
+    g_alibi_n = n;
+}
+
+/* The ALiBi paper's head slopes for n heads: for n a power of two, the
+ * geometric sequence whose first term and ratio are both 2^(-8/n); otherwise
+ * the slopes of the largest power of two m below n, followed by the first
+ * n - m terms at even positions (0, 2, 4, ...) of the sequence for 2m. */
+static double alibi_geometric(int n, int k)
+{
+    return pow(2.0, -8.0 * (double)(k + 1) / (double)n);
+}
+
+void oracle_alibi_slopes(int n, double *out)
+{
+    int m = 1;
+    while (2 * m <= n) m *= 2;
+    for (int k = 0; k < m && k < n; ++k) out[k] = alibi_geometric(m, k);
+    for (int k = m; k < n; ++k) out[k] = alibi_geometric(2 * m, 2 * (k - m));
 }
 
 static double rope_theta(int i, int d, double base)
@@ -308,6 +347,7 @@ int oracle_attend(int num_req, int num_q_heads, int num_kv_heads, int head_dim,
     const double scale = softmax_scale > 0 ? softmax_scale : 1.0 / sqrt((double)d);
     const int64_t total_q = cu_q[num_req];
     const int64_t n_rows = n_sel >= 0 ? n_sel : total_q * Hq;
+    const int alibi = g_alibi_n == Hq;   /* linear position penalty in place of RoPE */
     int rc = OR_OK;
 
     for (int r = 0; r < num_req; ++r) {
@@ -340,7 +380,10 @@ int oracle_attend(int num_req, int num_q_heads, int num_kv_heads, int head_dim,
                     double x[1024];
                     if (d > 1024) { rc = OR_EINVAL; continue; }
                     for (int i = 0; i < d; ++i) x[i] = oracle_bf16_to_f64(kr[i]);
-                    oracle_rope(x, d, rope_base, P[t], K + ((size_t)t * Hkv + h) * d);
+                    if (alibi)
+                        memcpy(K + ((size_t)t * Hkv + h) * d, x, sizeof(double) * (size_t)d);
+                    else
+                        oracle_rope(x, d, rope_base, P[t], K + ((size_t)t * Hkv + h) * d);
                     for (int i = 0; i < d; ++i) V[((size_t)t * Hkv + h) * d + i] = oracle_bf16_to_f64(vr[i]);
                 }
             }
@@ -361,7 +404,10 @@ int oracle_attend(int num_req, int num_q_heads, int num_kv_heads, int head_dim,
             int64_t p = q_pos[q];
             double xq[1024], qr[1024];
             for (int k = 0; k < d; ++k) xq[k] = oracle_bf16_to_f64(q_raw[((size_t)q * Hq + h) * d + k]);
-            oracle_rope(xq, d, rope_base, p, qr);
+            if (alibi)
+                memcpy(qr, xq, sizeof(double) * (size_t)d);
+            else
+                oracle_rope(xq, d, rope_base, p, qr);
             double *s = (double *)malloc(sizeof(double) * (size_t)(kv_len > 0 ? kv_len : 1));
             double m = -INFINITY;
             for (int64_t u = 0; u < kv_len; ++u) {
@@ -370,6 +416,7 @@ int oracle_attend(int num_req, int num_q_heads, int num_kv_heads, int head_dim,
                     double acc = 0.0;
                     for (int k = 0; k < d; ++k) acc += qr[k] * kk[k];
                     s[u] = acc * scale;
+                    if (alibi) s[u] -= g_alibi[h] * (double)(p - P[u]);
                     if (s[u] > m) m = s[u];
                 } else {
                     s[u] = -INFINITY;

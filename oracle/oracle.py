@@ -90,6 +90,10 @@ def _bind(lib) -> None:
         ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_double, _u16p, _i32p, _u16p]
     lib.oracle_set_rope_theta.restype = None
     lib.oracle_set_rope_theta.argtypes = [_f64p, ctypes.c_int]
+    lib.oracle_set_alibi.restype = None
+    lib.oracle_set_alibi.argtypes = [_f64p, ctypes.c_int]
+    lib.oracle_alibi_slopes.restype = None
+    lib.oracle_alibi_slopes.argtypes = [ctypes.c_int, _f64p]
     lib.oracle_llama31_theta.restype = None
     lib.oracle_llama31_theta.argtypes = [ctypes.c_double, ctypes.c_int, ctypes.c_double, ctypes.c_double,
                                          ctypes.c_double, ctypes.c_double, _f64p]
@@ -119,6 +123,31 @@ class _Theta:
         if self.theta is not None:
             self.lib.oracle_set_rope_theta(ctypes.cast(None, _f64p), 0)
         return False
+
+
+class _Alibi:
+    """Sets the oracle's ALiBi slopes (one per query head) for one call (None: RoPE)."""
+
+    def __init__(self, lib, slopes):
+        self.lib = lib
+        self.slopes = None if slopes is None else _c(slopes, np.float64)
+
+    def __enter__(self):
+        if self.slopes is not None:
+            self.lib.oracle_set_alibi(_p(self.slopes, _f64p), int(self.slopes.size))
+        return self
+
+    def __exit__(self, *exc):
+        if self.slopes is not None:
+            self.lib.oracle_set_alibi(ctypes.cast(None, _f64p), 0)
+        return False
+
+
+def alibi_slopes(n_heads: int, lib=None) -> np.ndarray:
+    """The ALiBi paper's head slopes for n_heads heads (the oracle's own computation)."""
+    out = np.empty(n_heads, np.float64)
+    (lib or _load()).oracle_alibi_slopes(int(n_heads), _p(out, _f64p))
+    return out
 
 
 def llama31_theta(base: float = 500000.0, d: int = 128, factor: float = 8.0, low_factor: float = 1.0,
@@ -218,12 +247,14 @@ def expand_table(words, blk_meta, num_blocks: int):
 
 def attend(*, num_q_heads: int, num_kv_heads: int, rope_base: float, q_raw, cu_q, q_pos,
            seg_indptr, seg_src, seg_off, seg_len, k_tok, v_tok, sel_q=None, sel_h=None,
-           softmax_scale: float = 0.0, want_scores: bool = False, lib=None, rope_theta=None):
+           softmax_scale: float = 0.0, want_scores: bool = False, lib=None, rope_theta=None,
+           alibi_slopes=None):
     """Materialised causal GQA attention in fp64.
 
     q_raw: uint16 [total_q, Hq, d]; k_tok, v_tok: uint16 [n_store, Hkv, d].
     Returns out [n_rows, d] float64 (rows: the selection, or every (q, h) in
     q-major order) and, if want_scores, scores [n_rows, max_kv_len].
+    alibi_slopes (one per query head) replaces RoPE by the linear ALiBi penalty.
     """
     q_raw = _c(q_raw, np.uint16)
     k_tok = _c(k_tok, np.uint16)
@@ -257,7 +288,9 @@ def attend(*, num_q_heads: int, num_kv_heads: int, rope_base: float, q_raw, cu_q
         scores = None
         sp = ctypes.cast(None, _f64p)
     lib = lib or _load()
-    with _Theta(lib, rope_theta):
+    if alibi_slopes is not None and len(alibi_slopes) != num_q_heads:
+        raise ValueError("alibi_slopes needs one slope per query head")
+    with _Theta(lib, rope_theta), _Alibi(lib, alibi_slopes):
         rc = lib.oracle_attend(
             int(num_req), int(num_q_heads), int(num_kv_heads), int(d), float(rope_base),
             float(softmax_scale), _p(q_raw, _u16p), _p(cu_q, _i32p), _p(q_pos, _i32p),

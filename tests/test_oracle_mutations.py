@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 
 import oracle
-from tests.test_oracle_pins import _adversarial_case, _brute_scores_and_out
+from tests.test_oracle_pins import ALIBI_PINS, _adversarial_case, _brute_scores_and_out
 
 SRC = os.path.join(os.path.dirname(oracle.lib_path()), "..", "lazy_oracle.c")
 
@@ -43,6 +43,39 @@ def test_planted_mistake_is_caught(name, tmp_path):
     assert not np.allclose(out, ref, rtol=1e-9, atol=1e-10), f"mutation {name} was not detected"
     # and the unmutated oracle passes the same check
     assert np.allclose(oracle.attend(**case.oracle_kwargs()), ref, rtol=1e-12, atol=1e-13)
+
+
+ALIBI_MUTATIONS = {
+    "alibi_sign": ("s[u] -= g_alibi[h] * (double)(p - P[u]);", "s[u] += g_alibi[h] * (double)(p - P[u]);"),
+    "alibi_kv_head_slope": ("s[u] -= g_alibi[h] * (double)(p - P[u]);", "s[u] -= g_alibi[kvh] * (double)(p - P[u]);"),
+    "alibi_no_key_position": ("s[u] -= g_alibi[h] * (double)(p - P[u]);", "s[u] -= g_alibi[h] * (double)(p);"),
+    "alibi_query_still_rotated": ("if (alibi)\n                memcpy(qr, xq", "if (0)\n                memcpy(qr, xq"),
+    "alibi_slopes_odd_terms": ("alibi_geometric(2 * m, 2 * (k - m))", "alibi_geometric(2 * m, 2 * (k - m) + 1)"),
+    "alibi_slopes_exponent": ("-8.0 * (double)(k + 1)", "-8.0 * (double)k"),
+}
+
+
+def _alibi_pins_fail(lib) -> list[str]:
+    failed = []
+    for pin in ALIBI_PINS:
+        try:
+            pin(lib=lib)
+        except AssertionError:
+            failed.append(pin.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(ALIBI_MUTATIONS))
+def test_planted_alibi_mistake_is_caught(name, tmp_path):
+    old, new = ALIBI_MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    mut = tmp_path / "mut.c"
+    mut.write_text(src.replace(old, new))
+    so = tmp_path / "mut.so"
+    subprocess.check_call(["gcc", "-O1", "-std=gnu99", "-fPIC", "-shared", "-o", str(so), str(mut), "-lm"])
+    assert _alibi_pins_fail(oracle.load_library(str(so))), f"mutation {name} was not detected"
+    assert not _alibi_pins_fail(None)
 
 
 # ----------------------------------------------------------------------------- reference block cache

@@ -15,7 +15,13 @@ a re-typed copy of its formulas:
   * softmax invariants (constant values reproduce themselves, a single
     visible key returns its value exactly, no visible key gives zeros);
   * bf16 rounding against torch's float32 -> bf16 conversion and hand ties;
-  * the table-word codec against hand-computed words.
+  * the table-word codec against hand-computed words;
+  * ALiBi (Key Contributions: the method extends to other relative
+    encodings): the default head slopes against values derived by hand from
+    the ALiBi paper's rule; with identical keys every score is the same up to
+    the bias, so each head's output is a geometric-weight average with a
+    closed form; equality with torch's float64 SDPA given the bias as an
+    additive mask on contiguous placements; shift invariance.
 """
 import numpy as np
 import pytest
@@ -326,3 +332,96 @@ def test_rope_with_a_table_is_relative_and_default_table_matches():
     np.testing.assert_array_equal(oracle.rope(q, 4321, 500000.0, theta=dflt), oracle.rope(q, 4321, 500000.0))
     # and the scaled table really changes long-wavelength components
     assert not np.allclose(oracle.rope(q, 4321, 500000.0, theta=th), oracle.rope(q, 4321, 500000.0))
+
+
+# --------------------------------------------------------------------------- ALiBi
+def alibi_pin_slopes_by_hand(lib=None):
+    # the rule: n a power of two -> 2^(-8k/n), k = 1..n; otherwise the 2^m < n slopes, then the
+    # even-position terms of the 2^(m+1) sequence
+    want = {1: [-8.0], 2: [-4.0, -8.0], 8: list(-np.arange(1.0, 9.0)), 6: [-2.0, -4.0, -6.0, -8.0, -1.0, -3.0],
+            12: [-1.0, -2.0, -3.0, -4.0, -5.0, -6.0, -7.0, -8.0, -0.5, -1.5, -2.5, -3.5]}
+    for n, e in want.items():
+        np.testing.assert_allclose(oracle.alibi_slopes(n, lib=lib), 2.0 ** np.array(e), rtol=1e-15, atol=0)
+
+
+def alibi_pin_geometric_weights(lib=None):
+    # every key the same vector: q.k is one constant per (query, head), so the weights are
+    # exp(-m_h (p - t)) / sum, a geometric sequence in the distance; component 0 of the output is
+    # then the weighted mean of the values' component 0 over the visible keys
+    case = _adversarial_case(hq=4, hkv=2)
+    case.k_tok[:] = case.k_tok[0:1]
+    slopes = np.array([0.5, 0.125, 0.03, 0.9])
+    out = oracle.attend(**case.oracle_kwargs(), alibi_slopes=slopes, lib=lib)
+    G = case.hq // case.hkv
+    i = 0
+    for r in range(case.cu_q.size - 1):
+        keys = [(case.seg_src[g] + j, case.seg_off[g] + j)
+                for g in range(case.seg_indptr[r], case.seg_indptr[r + 1]) for j in range(case.seg_len[g])]
+        for q in range(case.cu_q[r], case.cu_q[r + 1]):
+            p = int(case.q_pos[q])
+            for h in range(case.hq):
+                vis = [(row, pos) for row, pos in keys if pos <= p]
+                if not vis:
+                    assert np.all(out[i] == 0)
+                else:
+                    w = np.array([np.exp(-slopes[h] * (p - pos)) for _, pos in vis])
+                    v0 = np.array([bits_to_f64(case.v_tok[row, h // G])[0] for row, _ in vis])
+                    np.testing.assert_allclose(out[i, 0], (w * v0).sum() / w.sum(), rtol=1e-12, atol=1e-13)
+                i += 1
+
+
+def alibi_pin_contiguous_equals_sdpa(lib=None):
+    lens = [9, 13, 6]
+    segs, row = [], 0
+    for o, L in zip(np.cumsum([0] + lens[:-1]), lens):
+        segs.append((row, int(o), L))
+        row += L
+    total = sum(lens)
+    qp = np.arange(total - 6, total)
+    hq, hkv = 6, 3
+    case = make_case(12, hq=hq, hkv=hkv, d=D, requests=[(segs, list(qp))])
+    slopes = oracle.alibi_slopes(hq, lib=lib)
+    out = oracle.attend(**case.oracle_kwargs(), alibi_slopes=slopes, lib=lib)
+    # no rotation; the bias as an additive float mask, -inf where the key is in the future
+    G = hq // hkv
+    K = torch.from_numpy(bits_to_f64(case.k_tok[:total])).permute(1, 0, 2).repeat_interleave(G, 0)
+    V = torch.from_numpy(bits_to_f64(case.v_tok[:total])).permute(1, 0, 2).repeat_interleave(G, 0)
+    Q = torch.from_numpy(bits_to_f64(case.q_raw)).permute(1, 0, 2)
+    dist = qp[:, None] - np.arange(total)[None, :]
+    bias = -slopes[:, None, None] * dist[None]
+    bias = np.where(dist[None] >= 0, bias, -np.inf)
+    ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=torch.from_numpy(bias))
+    np.testing.assert_allclose(out, ref.permute(1, 0, 2).reshape(-1, D).numpy(), rtol=1e-12, atol=1e-13)
+    # slopes of zero: plain causal attention without any positional encoding
+    out0 = oracle.attend(**case.oracle_kwargs(), alibi_slopes=np.zeros(hq), lib=lib)
+    ref0 = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=torch.from_numpy(dist >= 0))
+    np.testing.assert_allclose(out0, ref0.permute(1, 0, 2).reshape(-1, D).numpy(), rtol=1e-12, atol=1e-13)
+
+
+def alibi_pin_shift_invariance(lib=None):
+    case = _adversarial_case()
+    slopes = oracle.alibi_slopes(case.hq, lib=lib)
+    out0 = oracle.attend(**case.oracle_kwargs(), alibi_slopes=slopes, lib=lib)
+    for c in (1, 977, 12345):
+        kw = case.oracle_kwargs()
+        kw["seg_off"] = case.seg_off + c
+        kw["q_pos"] = case.q_pos + c
+        np.testing.assert_allclose(oracle.attend(**kw, alibi_slopes=slopes, lib=lib), out0, rtol=1e-10, atol=1e-11)
+
+
+ALIBI_PINS = [alibi_pin_slopes_by_hand, alibi_pin_geometric_weights, alibi_pin_contiguous_equals_sdpa,
+              alibi_pin_shift_invariance]
+
+
+@pytest.mark.parametrize("pin", ALIBI_PINS, ids=lambda f: f.__name__)
+def test_alibi(pin):
+    pin()
+
+
+def test_alibi_needs_one_slope_per_query_head_and_leaves_rope_calls_alone():
+    case = _adversarial_case()
+    with pytest.raises(ValueError):
+        oracle.attend(**case.oracle_kwargs(), alibi_slopes=np.ones(case.hq + 1))
+    a = oracle.attend(**case.oracle_kwargs())
+    oracle.attend(**case.oracle_kwargs(), alibi_slopes=np.ones(case.hq))
+    assert np.array_equal(oracle.attend(**case.oracle_kwargs()), a)
