@@ -16,7 +16,8 @@ a 512 MiB buffer outside the timed intervals.
 Also measured in the same run and reported in sub-objects:
   prefill     the causal prefill workload with 8B shapes (16 requests x 256
               query tokens over 10 documents), TFLOP/s over visible pairs;
-  comparison  the position-aware alternative on the same inputs:
+  comparison  the position-aware alternative on the same inputs (and the same attention with ALiBi
+              in place of RoPE, timing only):
               materialise re-rotated keys, then plain paged attention;
   e2e         the decode metric through the same C-ABI calls with the step's
               inputs copied from pinned host memory and the output copied back
@@ -53,9 +54,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TRAFFIC = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
     #     -k regex:decode_split -s 3 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu --no-compare --no-e2e
-    "decode_8b": {"sha": "1882d73735d88144", "bytes": 782188544 + 7172352},
+    "decode_8b": {"sha": "15c7ea765fb0e618", "bytes": 781579776 + 7021568},
     # the same with -k regex:prefill_tc
-    "prefill_8b": {"sha": "3eb263b89dd13961", "bytes": 305164032 + 27624704},
+    "prefill_8b": {"sha": "e766bd345ac84128", "bytes": 300506624 + 25670912},
 }
 
 
@@ -311,14 +312,16 @@ def run_ours(args):
         mat_total, _ = timed_steps(mat_step, args.steps, args.warmup, flush, world)
         torch.cuda.synchronize()
         lazy_vs_plain = float((ds.out.float() - ds.out_plain.float()).abs().max().item())
+        alibi_total = _time_alibi(ds, args, flush, world)
         result["comparison"] = {
             "lazy_decode_attn_ms": round(attn_avg, 5),
             "plain_decode_attn_ms": round(max_over_ranks(world, plain_total / args.steps), 5),
             "materialize_then_attend_ms": round(max_over_ranks(world, mat_total / args.steps), 5),
             "materialized_k_bytes": int(ds.k_mat.numel() * 2),
             "max_abs_lazy_minus_plain": lazy_vs_plain,
+            "alibi_decode_attn_ms": round(max_over_ranks(world, alibi_total / args.steps), 5),
         }
-        result["gpu_launches"] += 2 * args.steps + 3 * args.steps
+        result["gpu_launches"] += 2 * args.steps + 3 * args.steps + 2 * args.steps
 
     # ---------------------------------------------------------------- e2e through the public API
     if not args.no_e2e:
@@ -413,6 +416,22 @@ def run_e2e(ds, pool, step, dec_bytes, args, world):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
+def _time_alibi(ds, args, flush, world) -> float:
+    """The step's attention with ALiBi (the model's slopes for its query heads) in place of RoPE,
+    on the same pool and inputs: the cost of the other relative encoding.  Timing only (the pool
+    holds RoPE keys, so the values are not compared here; the parity tests check ALiBi)."""
+    import dataclasses
+
+    from position_agnostic_paged_b200.rope import alibi_slopes
+    rope_cfg = ds.cfg
+    ds.cfg = dataclasses.replace(rope_cfg, alibi_slopes=alibi_slopes(rope_cfg.num_q_heads))
+    try:
+        total, _ = timed_steps(lambda ev: ds.attend(out=ds.out_plain), args.steps, args.warmup, flush, world)
+    finally:
+        ds.cfg = rope_cfg
+    return total
+
+
 def run_prefill(args, world, peaks, peak_src, flush):
     import torch
 
@@ -466,11 +485,13 @@ def run_prefill(args, world, peaks, peak_src, flush):
             "materialized_k_bytes": int(ds.k_mat.numel() * 2),
             "max_abs_lazy_minus_plain": float((ds.out.float() - ds.out_plain.float()).abs().max().item()),
         }
+        alibi_total = _time_alibi(ds, args, flush, world)
+        comparison["alibi_prefill_attn_ms"] = round(max_over_ranks(world, alibi_total / args.steps), 5)
     # attention launches per call: the prefill kernel, plus the combine kernel when the workspace
     # lets the last wave's units run split
     per_call = 2 if ds.workspace.numel() >= 16 and la.prefill_workspace_bytes(
         ds.cfg, step.num_req, step.total_q, ds.max_q, ds.max_words) > 0 else 1
-    launches = (1 + per_call) * args.steps + ((per_call + 1 + per_call) * args.steps if comparison else 0)
+    launches = (1 + per_call) * args.steps + ((per_call + 1 + per_call + per_call) * args.steps if comparison else 0)
     return {
         "_launches": launches,
         "workload": "prefill_8b: Llama-3.1-8B shapes, 16 requests x 256 causal query tokens over 10 Zipf(1.0) "
@@ -485,6 +506,15 @@ def run_prefill(args, world, peaks, peak_src, flush):
     }
 
 
+def _pf_calls(ds) -> int:
+    """Launches of one prefill attention call: the kernel, and the combine kernel when the
+    workspace lets the last wave's units run split."""
+    from position_agnostic_paged_b200 import lazy_attn as la
+    st = ds.step
+    return 2 if ds.workspace.numel() >= 16 and la.prefill_workspace_bytes(
+        ds.cfg, st.num_req, st.total_q, ds.max_q, ds.max_words) > 0 else 1
+
+
 def run_extended(args, world, peaks, peak_src, flush):
     """Decode 70B shapes (Zipf 1.2 and uniform popularity) and the mixed 8B serving
     step (32 prefill chunks + 192 decodes, 1 GiB pool; GQA and MQA): per step
@@ -493,7 +523,7 @@ def run_extended(args, world, peaks, peak_src, flush):
 
     from position_agnostic_paged_b200 import accounting
     from position_agnostic_paged_b200 import workloads as W
-    from position_agnostic_paged_b200.runner import DevicePool, DeviceStep
+    from position_agnostic_paged_b200.runner import DevicePool, DeviceStep, mixed_attend
 
     out = {}
     for name in ("decode_70b", "decode_70b_uniform", "mixed_8b", "mixed_8b_mqa"):
@@ -501,6 +531,7 @@ def run_extended(args, world, peaks, peak_src, flush):
         wl = W.make(name)
         pool = DevicePool(wl).setup()
         entry = {"unique_docs": wl.info["unique_docs_used"], "pool_blocks": wl.num_blocks}
+        kept = {}
         for step in wl.steps:
             ds = DeviceStep(pool, step)
             _prepare_step_writes(ds)
@@ -526,7 +557,26 @@ def run_extended(args, world, peaks, peak_src, flush):
                 entry["prefill"] = {"requests": step.num_req, "flops": f, "attn_ms": round(attn, 5),
                                     "TFLOP/s": round(tf, 1),
                                     "frac_of_bf16_peak": round(tf / peaks.get("bf16_tflops", 1590.0), 4)}
-            del ds
+            kept[step.kind] = ds
+        if "prefill" in kept and "decode" in kept:
+            # the whole serving step: the two attention calls back to back on one stream, and the
+            # same two batches in one lazy_mixed_attn call (decode on the side stream)
+            pf, dc = kept["prefill"], kept["decode"]
+
+            def seq(ev):
+                pf.attend()
+                dc.attend()
+
+            def mixed(ev):
+                mixed_attend(pf, dc)
+
+            seq_total, _ = timed_steps(seq, args.steps, args.warmup, flush, world)
+            mix_total, _ = timed_steps(mixed, args.steps, args.warmup, flush, world)
+            entry["step"] = {"sequential_ms": round(max_over_ranks(world, seq_total / args.steps), 5),
+                             "lazy_mixed_attn_ms": round(max_over_ranks(world, mix_total / args.steps), 5)}
+            launches_extra = (_pf_calls(pf) + 2) * 2 * args.steps
+            entry["step"]["gpu_launches"] = launches_extra
+        del kept, ds
         if pool.status() != 0:
             raise SystemExit(f"device status {pool.status()} in {name}")
         del pool

@@ -83,6 +83,18 @@ typedef struct lazy_attn_cfg {
      * (position difference) x theta_i.  The pages name other relative
      * encodings as within reach of the method but fix no table. */
     const double *rope_theta;
+    /* Optional: ALiBi in place of RoPE (ABI version 102).  NULL selects RoPE.
+     * Otherwise num_q_heads slopes m_h (num_q_heads <= 128, else
+     * LAZY_ESHAPE; each finite, else LAZY_EINVAL), read during the call only.
+     * Nothing is rotated: lazy_kv_write stores keys exactly as given, and the
+     * score of query head h at position p for the key at o + j gets
+     * -m_h * (p - o - j), computed from the table word's offset and the
+     * block's local index in the kernel, like the rotation angle of the RoPE
+     * path ([CON] lists ALiBi among the encodings the method extends to).
+     * The stored keys then carry no position at all, so the materialisation
+     * and plain comparison entry points refuse ALiBi (LAZY_EINVAL).  With
+     * ALiBi set, rope_base and rope_theta are ignored. */
+    const double *alibi_slopes;
 } lazy_attn_cfg;
 
 /* Host-side return codes. */
@@ -90,7 +102,7 @@ enum {
     LAZY_OK = 0,
     LAZY_EINVAL = -1,     /* null pointer or negative count */
     LAZY_ERANGE = -2,     /* a table field overflows 17/15 bits, or a size is too large */
-    LAZY_ESHAPE = -3,     /* head_dim != 128, block_size != 16, bad head counts */
+    LAZY_ESHAPE = -3,     /* head_dim != 128, block_size != 16, bad head counts (ALiBi: Hq > 128) */
     LAZY_EWORKSPACE = -4, /* workspace smaller than the matching *_workspace_bytes() */
     LAZY_ECUDA = -5       /* a CUDA launch or driver call failed */
 };
@@ -199,6 +211,56 @@ int lazy_prefill_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int
                       const uint32_t *blk_meta, const uint16_t *k_pool, const uint16_t *v_pool,
                       int num_blocks, uint16_t *out, void *workspace, size_t ws_bytes, int *d_status,
                       void *stream);
+
+/* ---- one serving step: prefill chunks and decodes in one call ---- */
+
+/* The arguments of lazy_prefill_attn for one batch of prefill chunks. */
+typedef struct lazy_prefill_batch {
+    const uint16_t *q_raw;
+    const int32_t *cu_q;
+    const int32_t *q_pos0;
+    int num_req, total_q, max_q;
+    const uint32_t *table;
+    const int32_t *table_indptr;
+    int max_words;
+    uint16_t *out;
+    void *workspace;
+    size_t ws_bytes;
+} lazy_prefill_batch;
+
+/* The arguments of lazy_decode_attn for one batch of decodes. */
+typedef struct lazy_decode_batch {
+    const uint16_t *q_raw;
+    const int32_t *q_pos;
+    int num_req;
+    const uint32_t *table;
+    const int32_t *table_indptr;
+    int max_words;
+    uint16_t *out;
+    void *workspace;
+    size_t ws_bytes;
+} lazy_decode_batch;
+
+/* A serving step that holds both prefill chunks and decodes over one pool
+ * (the mixed batches of a continuous-batching engine, as in the vLLM setting
+ * of [RES]).  The results are exactly those of lazy_prefill_attn(prefill)
+ * and lazy_decode_attn(decode) (the same kernels on the same inputs); the
+ * difference is scheduling.  Both batches are validated on the host before
+ * anything is enqueued, so an error leaves nothing half-launched.  The
+ * prefill runs on `stream`; the decode runs on a side stream of the library
+ * (one per device, created at the first call, non-blocking), forked from
+ * `stream` before the prefill and joined back into it after the decode, so
+ * work enqueued on `stream` afterwards sees both outputs.  Launched after the
+ * prefill, the decode's CTAs take the SMs that the prefill's last wave
+ * leaves idle, and no launch gap separates the two kernels.  Either batch
+ * may be NULL or empty (then this is the plain call on `stream`).  The two
+ * workspaces must be distinct buffers (LAZY_EINVAL otherwise).  Calls are
+ * serialised on the host by a mutex.  The fork and join are event waits, so
+ * the call can be captured in a CUDA graph; make one call on the device before
+ * capturing (the side stream is created then). */
+int lazy_mixed_attn(const lazy_attn_cfg *cfg, const lazy_prefill_batch *prefill, const lazy_decode_batch *decode,
+                    const uint32_t *blk_meta, const uint16_t *k_pool, const uint16_t *v_pool, int num_blocks,
+                    int *d_status, void *stream);
 
 /* ---- comparison paths (the position-aware alternative the pages argue against) ---- */
 

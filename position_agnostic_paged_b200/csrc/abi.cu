@@ -18,7 +18,7 @@ using namespace lazy;
 
 namespace {
 
-constexpr int kVersion = 101;
+constexpr int kVersion = 102;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -85,14 +85,21 @@ int check_cfg(const lazy_attn_cfg *cfg) {
     if (cfg->rope_theta)
         for (int i = 0; i < 64; ++i)
             if (!std::isfinite(cfg->rope_theta[i]) || cfg->rope_theta[i] < 0.0) return LAZY_EINVAL;
+    if (cfg->alibi_slopes) {
+        if (cfg->num_q_heads > kMaxAlibiHeads) return LAZY_ESHAPE;
+        for (int h = 0; h < cfg->num_q_heads; ++h)
+            if (!std::isfinite(cfg->alibi_slopes[h])) return LAZY_EINVAL;
+    }
     return LAZY_OK;
 }
 
 void fill_rope(RopeTableHost &t, const lazy_attn_cfg *cfg) {
-    // theta_i for the rotate-half pairs (i, i + d/2): the caller's table, else base^(-2i/d)
+    // theta_i for the rotate-half pairs (i, i + d/2): the caller's table, else base^(-2i/d);
+    // under ALiBi all zero, so that every rotation (pool write, query) is exactly the identity
     for (int i = 0; i < 64; ++i)
-        t.theta[i] = cfg->rope_theta ? cfg->rope_theta[i]
-                                     : std::pow(static_cast<double>(cfg->rope_base), -2.0 * i / 128.0);
+        t.theta[i] = cfg->alibi_slopes ? 0.0
+                     : cfg->rope_theta ? cfg->rope_theta[i]
+                                       : std::pow(static_cast<double>(cfg->rope_base), -2.0 * i / 128.0);
 }
 
 float scale_log2(const lazy_attn_cfg *cfg) {
@@ -132,13 +139,16 @@ int attn_common(const lazy_attn_cfg *cfg, AttnParams &p, int num_req, const uint
     p.max_words = max_words;
     p.scale_log2 = scale_log2(cfg);
     fill_rope(p.rope, cfg);
+    p.alibi = cfg->alibi_slopes ? 1 : 0;
+    for (int h = 0; h < cfg->num_q_heads && cfg->alibi_slopes; ++h)
+        p.alibi_log2[h] = static_cast<float>(cfg->alibi_slopes[h] * 1.4426950408889634);   // log2(e)
     return LAZY_OK;
 }
 
 int decode_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *q_pos, int num_req,
                 const uint32_t *table, const int32_t *table_indptr, int max_words, const uint32_t *blk_meta,
                 const uint16_t *k_src, int64_t k_rows, const uint16_t *v_pool, int num_blocks, uint16_t *out,
-                void *workspace, size_t ws_bytes, int *d_status, void *stream, bool plain) {
+                void *workspace, size_t ws_bytes, int *d_status, void *stream, bool plain, bool dry = false) {
     AttnParams p;
     int rc = attn_common(cfg, p, num_req, table, table_indptr, max_words, blk_meta, v_pool, num_blocks, out,
                          d_status);
@@ -146,12 +156,14 @@ int decode_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *
     if (num_req == 0) return LAZY_OK;
     if (!q_raw || !q_pos || !k_src) return LAZY_EINVAL;
     if (max_words == 0 || num_blocks == 0 || k_rows == 0) {
+        if (dry) return LAZY_OK;
         // nothing can be visible: every output row is zero
         return launch_rc(cudaMemsetAsync(out, 0, static_cast<size_t>(num_req) * p.hq * 128 * 2,
                                          static_cast<cudaStream_t>(stream)));
     }
     const size_t need = decode_ws(cfg, num_req, max_words);
     if (!workspace || ws_bytes < need) return LAZY_EWORKSPACE;
+    if (dry) return LAZY_OK;
     const DecodePlan pl = decode_plan(num_req, cfg->num_kv_heads, max_words);
     p.q_raw = q_raw;
     p.q_pos = q_pos;
@@ -173,9 +185,7 @@ int prefill_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t 
                  int num_req, int total_q, int max_q, const uint32_t *table, const int32_t *table_indptr,
                  int max_words, const uint32_t *blk_meta, const uint16_t *k_src, int64_t k_rows,
                  const uint16_t *v_pool, int num_blocks, uint16_t *out, void *workspace, size_t ws_bytes,
-                 int *d_status, void *stream, bool plain) {
-    (void)workspace;
-    (void)ws_bytes;
+                 int *d_status, void *stream, bool plain, bool dry = false) {
     AttnParams p;
     int rc = attn_common(cfg, p, num_req, table, table_indptr, max_words, blk_meta, v_pool, num_blocks, out,
                          d_status);
@@ -185,6 +195,7 @@ int prefill_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t 
     if (!q_raw || !cu_q || !q_pos0 || !k_src) return LAZY_EINVAL;
     if (static_cast<int64_t>(max_q) * p.group > (int64_t(1) << 30)) return LAZY_ERANGE;
     if (max_words == 0 || num_blocks == 0 || k_rows == 0) {
+        if (dry) return LAZY_OK;
         return launch_rc(cudaMemsetAsync(out, 0, static_cast<size_t>(total_q) * p.hq * 128 * 2,
                                          static_cast<cudaStream_t>(stream)));
     }
@@ -196,6 +207,7 @@ int prefill_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t 
     p.pf_mtiles = static_cast<int>((static_cast<int64_t>(max_q) * p.group + kPrefillRows - 1) / kPrefillRows);
     const long long units = static_cast<long long>(p.pf_mtiles) * p.hkv * num_req;
     if (units > (1LL << 30)) return LAZY_ERANGE;
+    if (dry) return LAZY_OK;
     int nsplit = prefill_split_units(units, sm_count());
     if (!workspace || ws_bytes < prefill_split_bytes(nsplit)) nsplit = 0;
     p.pf_nsplit = nsplit;
@@ -211,6 +223,37 @@ int prefill_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t 
         return LAZY_ECUDA;
     // each request writes exactly its own query tokens' rows
     return launch_rc(launch_prefill_tc(tk, tv, tk8, tv8, p, plain, static_cast<cudaStream_t>(stream)));
+}
+
+// The side stream of lazy_mixed_attn and its fork/join events, one set per device, created at
+// first use and kept for the life of the process.  g_mixed_mu also serialises the host-side
+// enqueue sequence of lazy_mixed_attn, so that each fork and join wait sees its own record.
+constexpr int kMaxMixedDevices = 64;
+struct MixedSide {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+MixedSide g_mixed[kMaxMixedDevices];
+std::mutex g_mixed_mu;
+
+int mixed_side(MixedSide **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxMixedDevices) return LAZY_ECUDA;
+    MixedSide &m = g_mixed[dev];
+    if (!m.stream) {
+        if (cudaStreamCreateWithFlags(&m.stream, cudaStreamNonBlocking) != cudaSuccess) {
+            m.stream = nullptr;
+            return LAZY_ECUDA;
+        }
+        if (cudaEventCreateWithFlags(&m.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&m.join, cudaEventDisableTiming) != cudaSuccess) {
+            cudaStreamDestroy(m.stream);
+            m.stream = nullptr;
+            return LAZY_ECUDA;
+        }
+    }
+    *out = &m;
+    return LAZY_OK;
 }
 
 }  // namespace
@@ -301,10 +344,69 @@ int lazy_prefill_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int
                         k_pool, rows, v_pool, num_blocks, out, workspace, ws_bytes, d_status, stream, false);
 }
 
+int lazy_mixed_attn(const lazy_attn_cfg *cfg, const lazy_prefill_batch *pf, const lazy_decode_batch *dc,
+                    const uint32_t *blk_meta, const uint16_t *k_pool, const uint16_t *v_pool, int num_blocks,
+                    int *d_status, void *stream) {
+    const bool has_pf = pf && pf->num_req > 0, has_dc = dc && dc->num_req > 0;
+    if (has_pf && has_dc && pf->workspace && dc->workspace && pf->workspace == dc->workspace) return LAZY_EINVAL;
+    if (cfg && check_cfg(cfg) == LAZY_OK && (has_pf || has_dc) && num_blocks > 0 && !k_pool) return LAZY_EINVAL;
+    const int64_t rows = cfg ? static_cast<int64_t>(num_blocks) * (cfg->num_kv_heads > 0 ? cfg->num_kv_heads : 0) * 16 : 0;
+    // both batches are checked before anything is enqueued
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (has_pf) {
+        rc = prefill_impl(cfg, pf->q_raw, pf->cu_q, pf->q_pos0, pf->num_req, pf->total_q, pf->max_q, pf->table,
+                          pf->table_indptr, pf->max_words, blk_meta, k_pool, rows, v_pool, num_blocks, pf->out,
+                          pf->workspace, pf->ws_bytes, d_status, stream, false, true);
+        if (rc) return rc;
+    }
+    if (has_dc) {
+        rc = decode_impl(cfg, dc->q_raw, dc->q_pos, dc->num_req, dc->table, dc->table_indptr, dc->max_words,
+                         blk_meta, k_pool, rows, v_pool, num_blocks, dc->out, dc->workspace, dc->ws_bytes, d_status,
+                         stream, false, true);
+        if (rc) return rc;
+    }
+    if (!has_pf || !has_dc) {
+        // one batch: the plain call on the caller's stream
+        if (has_pf)
+            return prefill_impl(cfg, pf->q_raw, pf->cu_q, pf->q_pos0, pf->num_req, pf->total_q, pf->max_q,
+                                pf->table, pf->table_indptr, pf->max_words, blk_meta, k_pool, rows, v_pool,
+                                num_blocks, pf->out, pf->workspace, pf->ws_bytes, d_status, stream, false);
+        if (has_dc)
+            return decode_impl(cfg, dc->q_raw, dc->q_pos, dc->num_req, dc->table, dc->table_indptr, dc->max_words,
+                               blk_meta, k_pool, rows, v_pool, num_blocks, dc->out, dc->workspace, dc->ws_bytes,
+                               d_status, stream, false);
+        return LAZY_OK;
+    }
+    std::lock_guard<std::mutex> lock(g_mixed_mu);
+    MixedSide *side = nullptr;
+    rc = mixed_side(&side);
+    if (rc) return rc;
+    const cudaStream_t main_s = static_cast<cudaStream_t>(stream);
+    // fork: the side stream starts after everything already on the caller's stream
+    if (cudaEventRecord(side->fork, main_s) != cudaSuccess || cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
+        return LAZY_ECUDA;
+    // prefill first, so that its CTAs (one per SM) are dispatched first; the decode's CTAs then
+    // take the SMs that its last, partial wave leaves free
+    const int rc_pf = prefill_impl(cfg, pf->q_raw, pf->cu_q, pf->q_pos0, pf->num_req, pf->total_q, pf->max_q,
+                                   pf->table, pf->table_indptr, pf->max_words, blk_meta, k_pool, rows, v_pool,
+                                   num_blocks, pf->out, pf->workspace, pf->ws_bytes, d_status, stream, false);
+    const int rc_dc = decode_impl(cfg, dc->q_raw, dc->q_pos, dc->num_req, dc->table, dc->table_indptr,
+                                  dc->max_words, blk_meta, k_pool, rows, v_pool, num_blocks, dc->out, dc->workspace,
+                                  dc->ws_bytes, d_status, side->stream, false);
+    // join, whatever happened: the caller's stream never runs ahead of the side stream's work
+    const bool joined = cudaEventRecord(side->join, side->stream) == cudaSuccess &&
+                        cudaStreamWaitEvent(main_s, side->join, 0) == cudaSuccess;
+    if (rc_pf) return rc_pf;
+    if (rc_dc) return rc_dc;
+    return joined ? LAZY_OK : LAZY_ECUDA;
+}
+
 int lazy_materialize_k(const lazy_attn_cfg *cfg, const uint32_t *table, int total_words, const uint32_t *blk_meta,
                        const uint16_t *k_pool, int num_blocks, uint16_t *k_mat, int *d_status, void *stream) {
     int rc = check_cfg(cfg);
     if (rc) return rc;
+    if (cfg->alibi_slopes) return LAZY_EINVAL;   // ALiBi keys carry no position to materialise
     if (total_words < 0 || num_blocks < 0) return LAZY_EINVAL;
     if (static_cast<uint32_t>(num_blocks) > LAZY_MAX_BLOCKS) return LAZY_ERANGE;
     if (total_words == 0) return LAZY_OK;
@@ -327,7 +429,7 @@ int lazy_plain_decode_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, cons
                            const uint32_t *blk_meta, const uint16_t *k_mat, int total_words, const uint16_t *v_pool,
                            int num_blocks, uint16_t *out, void *workspace, size_t ws_bytes, int *d_status,
                            void *stream) {
-    if (total_words < 0) return LAZY_EINVAL;
+    if (total_words < 0 || (cfg && cfg->alibi_slopes)) return LAZY_EINVAL;
     if (cfg && check_cfg(cfg) == LAZY_OK && num_req > 0 && total_words > 0 && !k_mat) return LAZY_EINVAL;
     const int64_t rows = cfg ? static_cast<int64_t>(total_words) * (cfg->num_kv_heads > 0 ? cfg->num_kv_heads : 0) * 16 : 0;
     if (rows >= (int64_t(1) << 31)) return LAZY_ERANGE;
@@ -340,7 +442,7 @@ int lazy_plain_prefill_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, con
                             const int32_t *table_indptr, int max_words, const uint32_t *blk_meta,
                             const uint16_t *k_mat, int total_words, const uint16_t *v_pool, int num_blocks,
                             uint16_t *out, void *workspace, size_t ws_bytes, int *d_status, void *stream) {
-    if (total_words < 0) return LAZY_EINVAL;
+    if (total_words < 0 || (cfg && cfg->alibi_slopes)) return LAZY_EINVAL;
     if (cfg && check_cfg(cfg) == LAZY_OK && num_req > 0 && total_words > 0 && !k_mat) return LAZY_EINVAL;
     const int64_t rows = cfg ? static_cast<int64_t>(total_words) * (cfg->num_kv_heads > 0 ? cfg->num_kv_heads : 0) * 16 : 0;
     if (rows >= (int64_t(1) << 31)) return LAZY_ERANGE;

@@ -18,6 +18,10 @@
 // when G is 16 or 32.  Per-warp online-softmax states are merged in shared
 // memory; split partials (m, l, acc) go to the workspace and a second kernel
 // combines them (flash-decoding).
+//
+// ALiBi (p.alibi): the frequency table is zero, so the query "rotation" is the
+// identity and runs once; each score gets slope_h * (o + j - p) in log2 units,
+// with o + j from the table word and the block's local index, as the mask uses.
 #include <climits>
 #include <cstdlib>
 
@@ -55,6 +59,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
     __shared__ uint64_t full_bar[kDecodeStages], empty_bar[kDecodeStages];
     __shared__ uint32_t stage_word[kDecodeStages], stage_meta[kDecodeStages];
     __shared__ double theta_s[kHalfDim];
+    __shared__ float slope_s[32];   // ALiBi slope (log2 units) of head g of the group; 0 past G
 
     const int split = blockIdx.x, kvh = blockIdx.y, r = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -75,6 +80,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
         fence_barrier_init();
     }
     if (threadIdx.x < kHalfDim) theta_s[threadIdx.x] = p.rope.theta[threadIdx.x];
+    if (threadIdx.x < 32) slope_s[threadIdx.x] = (p.alibi && threadIdx.x < G) ? p.alibi_log2[kvh * G + threadIdx.x] : 0.f;
     __syncthreads();
 
     // per-thread softmax state for query heads (8*ht + 2c, 8*ht + 2c + 1)
@@ -149,6 +155,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
         }
         uint32_t qb[8][2];
         int cur_off = INT_MIN;
+        // ALiBi slopes of this thread's two score columns (heads 8*ht + 2c, 8*ht + 2c + 1)
+        const float sl0 = slope_s[8 * ht + 2 * c], sl1 = slope_s[8 * ht + 2 * c + 1];
         const uint32_t stage0 = smem_u32(stages);
         // ldmatrix lane roles
         const int mi = lane >> 3, li = lane & 7;
@@ -167,7 +175,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
             if (b < static_cast<uint32_t>(p.num_blocks)) {
                 const uint32_t meta = stage_meta[st];
                 const int off = word_offset(w);
-                const int off_rot = PLAIN ? 0 : off;
+                const int off_rot = PLAIN ? 0 : (p.alibi ? qpos : off);
                 if (off_rot != cur_off) {
                     // re-rotate the query by (q_pos - offset): pairs (i, i+64)
                     // live in k-steps s and s+4 of the same thread
@@ -201,8 +209,16 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
                     ldsm_x4(kbase + swz_offset(k_key, 16 * s + k_dc, kBlockTokens), a0, a1, a2, a3);
                     mma_bf16(sacc, a0, a1, a2, a3, qb[s][0], qb[s][1]);
                 }
-                // causal / validity mask for keys rr and rr + 8
                 const int j0 = meta_j0(meta), nv = meta_valid(meta);
+                if (p.alibi) {
+                    // slope * (key position - query position) for keys rr and rr + 8
+                    const float d0 = static_cast<float>(off + j0 + rr - qpos), d1 = d0 + 8.f;
+                    sacc[0] = fmaf(sl0, d0, sacc[0]);
+                    sacc[1] = fmaf(sl1, d0, sacc[1]);
+                    sacc[2] = fmaf(sl0, d1, sacc[2]);
+                    sacc[3] = fmaf(sl1, d1, sacc[3]);
+                }
+                // causal / validity mask for keys rr and rr + 8
                 const bool vis0 = rr < nv && off + j0 + rr <= qpos;
                 const bool vis1 = rr + 8 < nv && off + j0 + rr + 8 <= qpos;
                 if (!vis0) sacc[0] = sacc[1] = -INFINITY;

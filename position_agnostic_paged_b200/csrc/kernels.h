@@ -14,6 +14,8 @@ struct RopeTableHost {
     double theta[64];
 };
 
+constexpr int kMaxAlibiHeads = 128;   // query heads an ALiBi call may have
+
 struct KvWriteParams {
     const uint16_t *k_raw, *v_raw;
     const int32_t *slot, *local_j;
@@ -65,7 +67,9 @@ struct AttnParams {
     int pf_mtiles, pf_base, pf_nsplit;
     int k_rows, v_rows;              // rows (of 128 bf16) covered by the K and V tensor maps
     float scale_log2;            // softmax scale * log2(e)
-    RopeTableHost rope;
+    RopeTableHost rope;          // all zero under ALiBi: every rotation is the identity
+    int alibi;                   // 1: add alibi_log2[h] * (key position - query position) to each score
+    float alibi_log2[kMaxAlibiHeads];   // ALiBi slope of query head h, times log2(e)
 };
 
 // Decode split plan shared by the workspace query and the launch.

@@ -83,7 +83,8 @@ constexpr int B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_KROT = B_KEMPTY + kK
               B_ODONE = B_PFULL + 2, B_QFULL = B_ODONE + 2, B_DRAIN = B_QFULL + 1, kNumBars = B_DRAIN + 1;
 constexpr int kOffTheta = kOffBar + kNumBars * 8;
 constexpr int kOffMisc = kOffTheta + kHalfDim * 8;
-constexpr int kSmemUse = kOffMisc + 16;
+constexpr int kOffSlope = kOffMisc + 16;                    // ALiBi: slopes of the group's G heads
+constexpr int kSmemUse = kOffSlope + 32 * 4;
 constexpr size_t kTcSmem = kSmemUse + 1024;
 static_assert(kTcSmem <= 232448, "shared memory budget");
 static_assert(sizeof(TileInfo) == 80, "tile info layout");
@@ -142,15 +143,25 @@ __device__ __forceinline__ bool rot_all(bool ok) {
     return any_fail == 0;
 }
 
-template <bool PLAIN>
+// MODE: kLazy (keys from the pool, each K tile rotated by (o - P0)), kPlain (keys from a
+// materialised copy indexed by table position, queries rotated at absolute positions: the
+// comparison path), kAlibi (keys from the pool used as stored, nothing rotated, the ALiBi
+// bias slope_h * (o + j - p) added to each score before the mask).
+constexpr int kLazy = 0, kPlain = 1, kAlibi = 2;
+
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                  const __grid_constant__ CUtensorMap tmV,
                                                                  const __grid_constant__ CUtensorMap tmK8,
                                                                  const __grid_constant__ CUtensorMap tmV8,
                                                                  const AttnParams p) {
+    constexpr bool PLAIN = MODE == kPlain;   // K source indexed by table position
+    constexpr bool ROTK = MODE == kLazy;     // K tiles rotated in shared memory
+    constexpr bool ALIBI = MODE == kAlibi;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
+    float *slope_s = reinterpret_cast<float *>(sm + kOffSlope);
     TileInfo *info = reinterpret_cast<TileInfo *>(sm + kOffInfo);
     double *theta_s = reinterpret_cast<double *>(sm + kOffTheta);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc);
@@ -192,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         for (int i = 0; i < kInfoStages; ++i) {
             mbar_init(&bars[B_IFULL + i], 1);
-            mbar_init(&bars[B_IEMPTY + i], kInfoConsumers + (PLAIN ? 0 : 4));
+            mbar_init(&bars[B_IEMPTY + i], kInfoConsumers + (ROTK ? 4 : 0));
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bars[B_SFULL + t], 1);
@@ -206,6 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         fence_barrier_init();
     }
     if (threadIdx.x < kHalfDim) theta_s[threadIdx.x] = p.rope.theta[threadIdx.x];
+    if (ALIBI && threadIdx.x < G) slope_s[threadIdx.x] = p.alibi_log2[kvh * G + threadIdx.x];
     if (warp == 2) {
         tc::tmem_alloc(tmem_slot, 512);
         tc::tmem_relinquish();
@@ -360,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 mbar_arrive(&bars[B_IEMPTY + is]);
                 const int ks = j % kKStages;
                 // the plain path uses keys as loaded; the lazy path waits for their rotation
-                uint64_t *kready = PLAIN ? &bars[B_KFULL + ks] : &bars[B_KROT + ks];
+                uint64_t *kready = ROTK ? &bars[B_KROT + ks] : &bars[B_KFULL + ks];
                 if (!wait_or_abort(kready, (j / kKStages) & 1, abort_flag, p.d_status)) break;
                 tc::fence_after_sync();
                 const uint64_t kb = dK0 + static_cast<uint64_t>((ks * kTileBytes) >> 4);
@@ -401,6 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const int tok = row_ok ? R / G : tok_first;
         const int g = R % G;
         const int prow = pos0 + tok;
+        const float slope = ALIBI ? slope_s[g] : 0.f;
         const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
         // Q'_i = R(p_i - P0) q_i for this warpgroup's row tile (R(p_i) on the plain path):
         // thread (ch, rb) writes pairs 8ch..8ch+7 of rows rb + 16k; between rows rb + 16k and
@@ -491,10 +504,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             const bool full = (ti.flags & kFull) != 0;
             // visible keys of each 16-key block for this row: slots si < lim[k]
             int lim[kTileBlocks];
+            float bk[kTileBlocks];   // ALiBi: bias of slot 0 of block k, slope * (o + j0 - p); 0 otherwise
 #pragma unroll
             for (int k = 0; k < kTileBlocks; ++k) {
                 const int nv = k < n ? meta_valid(ti.meta[k]) : 0;
                 lim[k] = max(0, min(nv, prow - ti.off - meta_j0(ti.meta[k]) + 1));
+                bk[k] = ALIBI ? slope * static_cast<float>(ti.off + meta_j0(ti.meta[k]) - prow) : 0.f;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_IEMPTY + is]);
@@ -507,16 +522,39 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             tc::ld32(tS + lane_off + 64, *reinterpret_cast<uint32_t(*)[32]>(sv + 64));
             tc::ld32(tS + lane_off + 96, *reinterpret_cast<uint32_t(*)[32]>(sv + 96));
             tc::wait_ld();
+            if (ALIBI) {
+                // the in-block part of the bias, slope * s for slot s; the block part bk[k] enters
+                // the block maxima and the exponent's offset below (one op per score, not two)
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    sv[c] = __float_as_uint(fmaf(slope, static_cast<float>(c & 15), __uint_as_float(sv[c])));
+            }
             if (!full) {
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
                     sv[c] = (c & 15) < lim[c >> 4] ? sv[c] : 0xFF800000u;   // -inf: P = 0
             }
             float m0 = __uint_as_float(sv[0]), m1 = __uint_as_float(sv[1]);
+            if (ALIBI) {
+                // row max of (score + bias): per 16-key block, the block part added once
+                m0 = -INFINITY;
 #pragma unroll
-            for (int c = 2; c < 128; c += 2) {
-                m0 = fmaxf(m0, __uint_as_float(sv[c]));
-                m1 = fmaxf(m1, __uint_as_float(sv[c + 1]));
+                for (int k = 0; k < kTileBlocks; ++k) {
+                    float a = __uint_as_float(sv[16 * k]), b = __uint_as_float(sv[16 * k + 1]);
+#pragma unroll
+                    for (int c = 2; c < 16; c += 2) {
+                        a = fmaxf(a, __uint_as_float(sv[16 * k + c]));
+                        b = fmaxf(b, __uint_as_float(sv[16 * k + c + 1]));
+                    }
+                    m0 = fmaxf(m0, fmaxf(a, b) + bk[k]);
+                }
+                m1 = m0;
+            } else {
+#pragma unroll
+                for (int c = 2; c < 128; c += 2) {
+                    m0 = fmaxf(m0, __uint_as_float(sv[c]));
+                    m1 = fmaxf(m1, __uint_as_float(sv[c + 1]));
+                }
             }
             const float m_new = fmaxf(m_run, fmaxf(m0, m1));
             const bool need = m_new > m_run + kRescaleThreshold;
@@ -527,12 +565,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 l_run *= scale;
             }
             const float mu = m_run == -INFINITY ? 0.f : m_run;
+            // ALiBi: the exponent's offset per block, m - bk[k]
+            if (ALIBI) {
+#pragma unroll
+                for (int k = 0; k < kTileBlocks; ++k) bk[k] = mu - bk[k];
+            }
             // P = 2^(S - m) as bf16 pairs over the first 64 columns of S, row sum in fp32
             float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
             for (int e = 0; e < 64; ++e) {
-                const float p0 = fast_exp2(__uint_as_float(sv[2 * e]) - mu);
-                const float p1 = fast_exp2(__uint_as_float(sv[2 * e + 1]) - mu);
+                const float mo = ALIBI ? bk[e >> 3] : mu;
+                const float p0 = fast_exp2(__uint_as_float(sv[2 * e]) - mo);
+                const float p1 = fast_exp2(__uint_as_float(sv[2 * e + 1]) - mo);
                 ls0 += p0;
                 ls1 += p1;
                 sv[e] = pack_bf16(p0, p1);
@@ -621,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const int tid = threadIdx.x - 384;
         const int ch = tid & 7;
         const int rb = tid >> 3;
-        if (!PLAIN) {
+        if (ROTK) {
             int cur = INT_MIN;
             float kc[8], kn[8];
             for (int w = wbeg, j = 0; w < wend; ++j) {
@@ -707,10 +751,10 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(const AttnParams p
     reinterpret_cast<uint2 *>(p.out + (static_cast<size_t>(q0 + tok) * p.hq + kvh * G + g) * kHeadDim)[lane] = u;
 }
 
-template <bool PLAIN>
+template <int MODE>
 cudaError_t launch_t(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8, const CUtensorMap &tv8,
                      const AttnParams &p, cudaStream_t s) {
-    auto kern = prefill_tc_kernel<PLAIN>;
+    auto kern = prefill_tc_kernel<MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
     if (e != cudaSuccess) return e;
     static_assert(kRows == kPrefillRows, "rows per CTA");
@@ -725,7 +769,8 @@ cudaError_t launch_t(const CUtensorMap &tk, const CUtensorMap &tv, const CUtenso
 
 cudaError_t launch_prefill_tc(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8,
                               const CUtensorMap &tv8, const AttnParams &p, bool plain, cudaStream_t s) {
-    return plain ? launch_t<true>(tk, tv, tk8, tv8, p, s) : launch_t<false>(tk, tv, tk8, tv8, p, s);
+    if (plain) return launch_t<kPlain>(tk, tv, tk8, tv8, p, s);
+    return p.alibi ? launch_t<kAlibi>(tk, tv, tk8, tv8, p, s) : launch_t<kLazy>(tk, tv, tk8, tv8, p, s);
 }
 
 }  // namespace lazy

@@ -27,6 +27,7 @@ EXPORTED = [
     "lazy_materialize_k", "lazy_plain_decode_attn", "lazy_plain_prefill_attn",
     "lazy_debug_decode_table", "lazy_decode_attn_noalloc", "lazy_decode_noalloc_capacity",
     "lazy_cache_create", "lazy_cache_destroy", "lazy_cache_access", "lazy_cache_contains", "lazy_cache_stats",
+    "lazy_mixed_attn",
 ]
 
 
@@ -39,13 +40,16 @@ class LazyAttnError(RuntimeError):
 class LazyAttnCfg(ctypes.Structure):
     _fields_ = [("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
                 ("block_size", ctypes.c_int), ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float),
-                ("rope_theta", ctypes.POINTER(ctypes.c_double))]
+                ("rope_theta", ctypes.POINTER(ctypes.c_double)),
+                ("alibi_slopes", ctypes.POINTER(ctypes.c_double))]
 
 
 @dataclass(frozen=True)
 class Cfg:
     """rope_theta: optional head_dim/2 RoPE frequencies (e.g. rope.llama31_theta()) in place of
-    rope_base^(-2i/head_dim)."""
+    rope_base^(-2i/head_dim).  alibi_slopes: optional num_q_heads ALiBi slopes (e.g.
+    rope.alibi_slopes(num_q_heads)) in place of RoPE: keys are stored as given and each score gets
+    -slope_h * (query position - key position)."""
     num_q_heads: int
     num_kv_heads: int
     rope_base: float = 500000.0
@@ -53,10 +57,17 @@ class Cfg:
     block_size: int = 16
     softmax_scale: float = 0.0
     rope_theta: tuple | None = None
+    alibi_slopes: tuple | None = None
 
     def c(self) -> LazyAttnCfg:
         st = LazyAttnCfg(self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
-                         float(self.rope_base), float(self.softmax_scale), None)
+                         float(self.rope_base), float(self.softmax_scale), None, None)
+        if self.alibi_slopes is not None:
+            if len(self.alibi_slopes) != self.num_q_heads:
+                raise ValueError("alibi_slopes needs one slope per query head")
+            sl = (ctypes.c_double * len(self.alibi_slopes))(*[float(x) for x in self.alibi_slopes])
+            st._alibi_keepalive = sl
+            st.alibi_slopes = ctypes.cast(sl, ctypes.POINTER(ctypes.c_double))
         if self.rope_theta is not None:
             arr = (ctypes.c_double * len(self.rope_theta))(*[float(x) for x in self.rope_theta])
             st._theta_keepalive = arr
@@ -66,6 +77,19 @@ class Cfg:
 
 _vp, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
 _cfgp = ctypes.POINTER(LazyAttnCfg)
+
+
+class PrefillBatch(ctypes.Structure):
+    """lazy_prefill_batch: the arguments of lazy_prefill_attn for one batch."""
+    _fields_ = [("q_raw", _vp), ("cu_q", _vp), ("q_pos0", _vp), ("num_req", _i), ("total_q", _i), ("max_q", _i),
+                ("table", _vp), ("table_indptr", _vp), ("max_words", _i), ("out", _vp), ("workspace", _vp),
+                ("ws_bytes", _sz)]
+
+
+class DecodeBatch(ctypes.Structure):
+    """lazy_decode_batch: the arguments of lazy_decode_attn for one batch."""
+    _fields_ = [("q_raw", _vp), ("q_pos", _vp), ("num_req", _i), ("table", _vp), ("table_indptr", _vp),
+                ("max_words", _i), ("out", _vp), ("workspace", _vp), ("ws_bytes", _sz)]
 
 
 def _load():
@@ -91,6 +115,8 @@ def _load():
         "lazy_debug_decode_table": (_i, [_vp, _i64, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
         "lazy_decode_attn_noalloc": (_i, [_cfgp, _vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
         "lazy_decode_noalloc_capacity": (_sz, []),
+        "lazy_mixed_attn": (_i, [_cfgp, ctypes.POINTER(PrefillBatch), ctypes.POINTER(DecodeBatch), _vp, _vp, _vp, _i,
+                                 _vp, _vp]),
         "lazy_cache_create": (_vp, [_i64]),
         "lazy_cache_destroy": (None, [_vp]),
         "lazy_cache_access": (_i, [_vp, ctypes.c_uint64, ctypes.c_int32, _vp]),
@@ -180,6 +206,36 @@ def prefill_attn(cfg: Cfg, q_raw, cu_q, q_pos0, max_q: int, table, table_indptr,
         int(max_q), _ptr(table), _ptr(table_indptr), int(max_words), _ptr(blk_meta), _ptr(k_pool),
         _ptr(v_pool), int(k_pool.shape[0]), _ptr(out), _ptr(workspace), ws_bytes, _ptr(d_status),
         _stream(stream)))
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size() if t is not None else 0
+
+
+def mixed_attn(cfg: Cfg, prefill: dict | None, decode: dict | None, blk_meta, k_pool, v_pool, d_status=None,
+               stream=None):
+    """One serving step with prefill chunks and decodes (lazy_mixed_attn): the results of
+    prefill_attn(**prefill) and decode_attn(**decode); the decode runs on the library's side stream,
+    forked from and joined back into `stream`.
+
+    prefill: dict(q_raw, cu_q, q_pos0, max_q, table, table_indptr, max_words, out, workspace);
+    decode: dict(q_raw, q_pos, table, table_indptr, max_words, out, workspace).  The two
+    workspaces must be distinct."""
+    c = cfg.c()
+    pf = dc = None
+    if prefill is not None:
+        b = prefill
+        pf = PrefillBatch(_ptr(b["q_raw"]), _ptr(b["cu_q"]), _ptr(b["q_pos0"]), int(b["q_pos0"].numel()),
+                          int(b["q_raw"].shape[0]), int(b["max_q"]), _ptr(b["table"]), _ptr(b["table_indptr"]),
+                          int(b["max_words"]), _ptr(b["out"]), _ptr(b.get("workspace")), _nbytes(b.get("workspace")))
+    if decode is not None:
+        b = decode
+        dc = DecodeBatch(_ptr(b["q_raw"]), _ptr(b["q_pos"]), int(b["q_pos"].numel()), _ptr(b["table"]),
+                         _ptr(b["table_indptr"]), int(b["max_words"]), _ptr(b["out"]), _ptr(b["workspace"]),
+                         _nbytes(b["workspace"]))
+    _check("lazy_mixed_attn", _lib.lazy_mixed_attn(
+        ctypes.byref(c), ctypes.byref(pf) if pf is not None else None, ctypes.byref(dc) if dc is not None else None,
+        _ptr(blk_meta), _ptr(k_pool), _ptr(v_pool), int(k_pool.shape[0]), _ptr(d_status), _stream(stream)))
 
 
 def materialize_k(cfg: Cfg, table, blk_meta, k_pool, k_mat, d_status=None, stream=None):

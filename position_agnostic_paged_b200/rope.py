@@ -1,4 +1,5 @@
-"""RoPE frequency tables for the configuration's optional `rope_theta`.
+"""Position-encoding tables for the configuration: RoPE frequencies (`rope_theta`) and ALiBi head
+slopes (`alibi_slopes`).
 
 The kernels take their rotation frequencies from one host table per call:
 theta_i = base^(-2i/d) by default, or any table passed as `Cfg.rope_theta`.
@@ -39,3 +40,21 @@ def llama31_theta(base: float = 500000.0, head_dim: int = 128, factor: float = 8
             w = (original_max_position / wavelength - low_freq_factor) / (high_freq_factor - low_freq_factor)
             out.append(w * f + (1.0 - w) * f / factor)
     return tuple(out)
+
+
+def alibi_slopes(num_heads: int) -> tuple[float, ...]:
+    """ALiBi head slopes (Press, Smith and Lewis, "Train Short, Test Long", 2022) for Cfg.alibi_slopes.
+
+    With n a power of two the slopes are r, r^2, ..., r^n for r = 2^(-8/n).  Any other head count
+    takes the slopes of the largest power of two p below it and tops them up with every second
+    slope (the 1st, 3rd, 5th, ...) of the 2p-head sequence.
+    """
+    def geometric(n):
+        r = 2.0 ** (-8.0 / n)
+        return [r ** (k + 1) for k in range(n)]
+
+    if num_heads <= 0:
+        raise ValueError("num_heads must be positive")
+    p = 1 << (num_heads.bit_length() - 1)
+    return tuple(geometric(p) + geometric(2 * p)[::2][: num_heads - p])
+

@@ -110,6 +110,16 @@ class DeviceStep:
                             self.table_indptr, self.max_words, p.blk_meta, p.k_pool, p.v_pool, out,
                             self.workspace, p.d_status, stream)
 
+    def batch(self) -> dict:
+        """This step's arguments as a lazy_mixed_attn batch."""
+        b = dict(q_raw=self.q_raw, table=self.table, table_indptr=self.table_indptr, max_words=self.max_words,
+                 out=self.out, workspace=self.workspace)
+        if self.step.kind == "decode":
+            b["q_pos"] = self.q_pos
+        else:
+            b.update(cu_q=self.cu_q, q_pos0=self.q_pos0, max_q=self.max_q)
+        return b
+
     def materialize(self, stream=None) -> None:
         p = self.pool
         la.materialize_k(self.cfg, self.table, p.blk_meta, p.k_pool, self.k_mat, p.d_status, stream)
@@ -128,3 +138,11 @@ class DeviceStep:
     def out_f64(self, out=None) -> np.ndarray:
         o = self.out if out is None else out
         return o.float().cpu().numpy().astype(np.float64).reshape(-1, self.pool.wl.d)
+
+
+def mixed_attend(prefill: DeviceStep, decode: DeviceStep, stream=None) -> None:
+    """One serving step over one pool: the prefill chunks and the decodes in one lazy_mixed_attn call."""
+    p = prefill.pool
+    assert decode.pool is p, "both batches must use the same pool"
+    la.mixed_attn(p.cfg, prefill.batch(), decode.batch(), p.blk_meta, p.k_pool, p.v_pool, p.d_status, stream)
+

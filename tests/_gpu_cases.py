@@ -26,10 +26,11 @@ def _i32(a, dev):
 
 class DeviceCase:
     def __init__(self, case, dev="cuda", extra_blocks: int = 0, scatter_seed: int | None = None,
-                 rope_theta=None):
+                 rope_theta=None, alibi_slopes=None):
         self.case = case
         self.cfg = la.Cfg(case.hq, case.hkv, rope_base=case.base,
-                          rope_theta=None if rope_theta is None else tuple(float(x) for x in rope_theta))
+                          rope_theta=None if rope_theta is None else tuple(float(x) for x in rope_theta),
+                          alibi_slopes=None if alibi_slopes is None else tuple(float(x) for x in alibi_slopes))
         docs = {}
         for g in range(case.seg_src.size):
             src, ln = int(case.seg_src[g]), int(case.seg_len[g])
@@ -123,6 +124,43 @@ class DeviceCase:
             la.prefill_attn(self.cfg, q, cu, p0, max_q, self.table, self.table_indptr, self.max_words,
                             self.blk_meta, self.k_pool, self.v_pool, out, ws, self.d_status)
         return out.float().cpu().numpy().astype(np.float64).reshape(-1, c.d)
+
+    def mixed_batches(self, n_prefill: int):
+        """Requests 0..n_prefill-1 as a prefill batch (contiguous query positions), the rest as a
+        decode batch (one query each), both over this case's pool and table (the batches index the
+        one table through slices of its row pointer)."""
+        c = self.case
+        n = c.cu_q.size - 1
+        cu = c.cu_q
+        tp = int(cu[n_prefill])
+        assert np.array_equal(np.diff(cu[n_prefill:]), np.ones(n - n_prefill)), "decode: one query per request"
+        pf_cu = cu[: n_prefill + 1]
+        q_pos0 = [int(c.q_pos[cu[r]]) if cu[r + 1] > cu[r] else 0 for r in range(n_prefill)]
+        max_q = int(np.diff(pf_cu).max())
+        pf = dict(q_raw=_u16(c.q_raw[:tp], self.dev), cu_q=_i32(pf_cu, self.dev), q_pos0=_i32(q_pos0, self.dev),
+                  max_q=max_q, table=self.table, table_indptr=self.table_indptr[: n_prefill + 1],
+                  max_words=self.max_words,
+                  out=torch.zeros((tp, c.hq, c.d), dtype=torch.bfloat16, device=self.dev),
+                  workspace=torch.empty(max(16, la.prefill_workspace_bytes(self.cfg, n_prefill, tp, max_q,
+                                                                           self.max_words)),
+                                        dtype=torch.uint8, device=self.dev))
+        nd = n - n_prefill
+        dc = dict(q_raw=_u16(c.q_raw[tp:], self.dev), q_pos=_i32(c.q_pos[tp:], self.dev), table=self.table,
+                  table_indptr=self.table_indptr[n_prefill:], max_words=self.max_words,
+                  out=torch.zeros((nd, c.hq, c.d), dtype=torch.bfloat16, device=self.dev),
+                  workspace=torch.empty(max(16, la.decode_workspace_bytes(self.cfg, nd, self.max_words)),
+                                        dtype=torch.uint8, device=self.dev))
+        return pf, dc
+
+    def mixed(self, pf, dc, stream=None):
+        la.mixed_attn(self.cfg, pf, dc, self.blk_meta, self.k_pool, self.v_pool, self.d_status, stream)
+
+    def separate(self, pf, dc):
+        la.prefill_attn(self.cfg, pf["q_raw"], pf["cu_q"], pf["q_pos0"], pf["max_q"], pf["table"],
+                        pf["table_indptr"], pf["max_words"], self.blk_meta, self.k_pool, self.v_pool, pf["out"],
+                        pf["workspace"], self.d_status)
+        la.decode_attn(self.cfg, dc["q_raw"], dc["q_pos"], dc["table"], dc["table_indptr"], dc["max_words"],
+                       self.blk_meta, self.k_pool, self.v_pool, dc["out"], dc["workspace"], self.d_status)
 
     def status(self) -> int:
         return int(self.d_status.item())

@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_strerror():
-    assert la.version() == 101
+    assert la.version() == 102
     for code in (0, -1, -2, -3, -4, -5):
         assert la.strerror(code) and la.strerror(code) != "unknown error"
 
@@ -88,3 +88,43 @@ def test_decode_workspace_sizes():
     # one (m, l, acc[128]) record of fp32 per (request, kv head, split, head in group)
     assert a % ((128 + 2) * 4 * 4) == 0
     assert la.decode_workspace_bytes(la.Cfg(32, 8, head_dim=64), 64, 261) == 0
+
+
+def test_alibi_validation_returns_before_launch():
+    sl = tuple([0.25] * 8)
+    assert _call_decode(la.Cfg(256, 8, alibi_slopes=tuple([0.1] * 256))) == la.LAZY_ESHAPE   # Hq > 128
+    assert _call_decode(la.Cfg(8, 2, alibi_slopes=(float("nan"),) + sl[1:])) == la.LAZY_EINVAL
+    assert _call_decode(la.Cfg(8, 2, alibi_slopes=(float("inf"),) + sl[1:])) == la.LAZY_EINVAL
+    c = la.Cfg(8, 2, alibi_slopes=sl).c()
+    # the stored keys carry no position: materialisation and the plain paths refuse ALiBi
+    assert la._lib.lazy_materialize_k(ctypes.byref(c), 1, 4, 1, 1, 8, 1, None, None) == la.LAZY_EINVAL
+    assert la._lib.lazy_plain_decode_attn(ctypes.byref(c), 1, 1, 2, 1, 1, 4, 1, 1, 8, 1, 8, 1, 1, 1 << 20,
+                                          None, None) == la.LAZY_EINVAL
+    assert la._lib.lazy_plain_prefill_attn(ctypes.byref(c), 1, 1, 1, 1, 4, 4, 1, 1, 4, 1, 1, 8, 1, 8, 1, 1,
+                                           1 << 20, None, None) == la.LAZY_EINVAL
+    with pytest.raises(ValueError):
+        la.Cfg(8, 2, alibi_slopes=sl[:4]).c()
+
+
+def test_alibi_slopes_helper_by_hand():
+    from position_agnostic_paged_b200.rope import alibi_slopes
+    np.testing.assert_allclose(alibi_slopes(8), 2.0 ** -np.arange(1.0, 9.0), rtol=1e-15, atol=0)
+    np.testing.assert_allclose(np.log2(alibi_slopes(12)), [-1, -2, -3, -4, -5, -6, -7, -8, -0.5, -1.5, -2.5, -3.5],
+                               rtol=0, atol=1e-13)
+    with pytest.raises(ValueError):
+        alibi_slopes(0)
+
+
+def test_mixed_step_validates_both_batches_before_launching():
+    c = la.Cfg(8, 2).c()
+    pf = la.PrefillBatch(1, 1, 1, 2, 8, 4, 1, 1, 4, 1, 1, 1 << 20)
+    same_ws = la.DecodeBatch(1, 1, 2, 1, 1, 4, 1, 1, 1 << 20)
+    small_ws = la.DecodeBatch(1, 1, 2, 1, 1, 4, 1, 2, 16)
+    call = lambda cfg, p, d: la._lib.lazy_mixed_attn(ctypes.byref(cfg), ctypes.byref(p) if p else None,
+                                                    ctypes.byref(d) if d else None, 1, 1, 1, 8, None, None)
+    assert call(c, pf, same_ws) == la.LAZY_EINVAL          # one workspace for both batches
+    assert call(c, pf, small_ws) == la.LAZY_EWORKSPACE     # the decode batch fails: nothing launched
+    assert call(la.Cfg(8, 3).c(), pf, small_ws) == la.LAZY_ESHAPE
+    assert call(c, None, None) == la.LAZY_OK              # nothing to do
+    bad_pf = la.PrefillBatch(1, 1, 1, 2, -1, 4, 1, 1, 4, 1, 1, 1 << 20)
+    assert call(c, bad_pf, la.DecodeBatch(1, 1, 2, 1, 1, 4, 1, 3, 1 << 20)) == la.LAZY_EINVAL

@@ -335,6 +335,148 @@ def test_kv_write_with_a_frequency_table():
     assert int(st.item()) == 0
 
 
+# ----------------------------------------------------------------------------- ALiBi
+def _alibi_slopes(hq):
+    """The product's and the oracle's ALiBi slopes: two independent computations of the ALiBi
+    paper's rule, which must agree."""
+    from position_agnostic_paged_b200 import rope as prope
+    sp = np.array(prope.alibi_slopes(hq))
+    so = oracle.alibi_slopes(hq)
+    np.testing.assert_allclose(sp, so, rtol=1e-14, atol=0)
+    return sp, so
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 2), (32, 8), (32, 1), (64, 8)])
+@pytest.mark.parametrize("kind", ["decode", "prefill", "prefill_unsplit"])
+def test_alibi_attention(kind, hq, hkv):
+    """ALiBi in place of RoPE: keys stored as given, the bias from the table word's offset and the
+    block's local index; gaps, a document at two offsets and partial blocks as in the RoPE cases."""
+    sp, so = _alibi_slopes(hq)
+    case = make_case(200 + hq + hkv, hq=hq, hkv=hkv, d=128, requests=_adv_requests(kind == "decode"))
+    dc = DeviceCase(case, alibi_slopes=sp)
+    ref = oracle.attend(**case.oracle_kwargs(), alibi_slopes=so)
+    tol = edge_max_abs(case)
+    assert np.abs(ref - oracle.attend(**case.oracle_kwargs())).max() > 3 * tol   # the encoding matters
+    got = dc.decode() if kind == "decode" else dc.prefill(split=kind == "prefill")
+    check(got, ref, max_abs=tol, what=f"{kind} G={hq // hkv} alibi")
+    assert dc.status() == 0
+
+
+@pytest.mark.parametrize("kind", ["decode", "prefill"])
+def test_alibi_long_context_and_full_tiles(kind):
+    """Positions near 31k, 8-block tiles of one document, a document reused at three offsets."""
+    sp, so = _alibi_slopes(32)
+    segs = [(0, 30000, 300), (300, 30400, 260), (0, 31000, 300), (0, 100, 300)]
+    qp = [31400] if kind == "decode" else list(range(31300, 31420))
+    case = make_case(62, hq=32, hkv=8, d=128, requests=[(segs, qp), ([(300, 0, 260)], [255] if kind == "decode"
+                                                                      else list(range(200, 260)))])
+    dc = DeviceCase(case, alibi_slopes=sp)
+    ref = oracle.attend(**case.oracle_kwargs(), alibi_slopes=so)
+    got = dc.decode() if kind == "decode" else dc.prefill()
+    check(got, ref, max_abs=edge_max_abs(case), what=f"{kind} alibi long")
+    assert dc.status() == 0
+
+
+def test_kv_write_under_alibi_stores_keys_as_given():
+    rng = np.random.default_rng(72)
+    hkv, d, nb, n = 4, 128, 30, 300
+    k = (rng.standard_normal((n, hkv, d)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    v = (rng.standard_normal((n, hkv, d)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    slot = rng.permutation(nb * 16)[:n].astype(np.int32)
+    local_j = (16 * rng.integers(0, 1875, n) + slot % 16).astype(np.int32)
+    cfg = la.Cfg(hkv * 2, hkv, alibi_slopes=tuple(_alibi_slopes(hkv * 2)[0]))
+    dev = "cuda"
+    kp = torch.zeros((nb, hkv, 16, d), dtype=torch.bfloat16, device=dev)
+    vp = torch.zeros_like(kp)
+    meta = torch.zeros(nb, dtype=torch.int32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    u16 = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    la.kv_write(cfg, u16(k), u16(v), torch.from_numpy(slot).to(dev), torch.from_numpy(local_j).to(dev),
+                kp, vp, meta, st)
+    gk = kp.view(torch.int16).cpu().numpy().view(np.uint16)
+    gv = vp.view(torch.int16).cpu().numpy().view(np.uint16)
+    for t in range(n):
+        b, s_ = divmod(int(slot[t]), 16)
+        assert np.array_equal(gk[b, :, s_], k[t]) and np.array_equal(gv[b, :, s_], v[t])
+    okp = np.zeros((nb, hkv, 16, d), np.uint16)
+    ometa = np.zeros(nb, np.uint32)
+    assert oracle.kv_write(k, v, slot, local_j, okp, okp.copy(), ometa, 500000.0) == 0
+    assert np.array_equal(meta.cpu().numpy().view(np.uint32), ometa)
+    assert int(st.item()) == 0
+
+
+# ----------------------------------------------------------------------------- mixed serving step
+def _mixed_case(hq=32, hkv=8):
+    segs = [(0, 0, 200), (300, 210, 130), (0, 400, 200)]
+    other = [(300, 0, 130), (500, 140, 37)]
+    reqs = [(segs, list(range(600, 700))), (other, list(range(177, 230))), ([(0, 5, 200)], list(range(205, 206))),
+            (segs, [650]), (other, [300]), ([(500, 0, 37)], [36]), (segs[:1], [1000])]
+    return make_case(81, hq=hq, hkv=hkv, d=128, requests=reqs)
+
+
+def _f64(t):
+    return t.float().cpu().numpy().astype(np.float64).reshape(-1, 128)
+
+
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (32, 1)])
+def test_mixed_step_equals_separate_calls_and_the_oracle(hq, hkv):
+    case = _mixed_case(hq, hkv)
+    dc_ = DeviceCase(case)
+    pf, dc = dc_.mixed_batches(3)
+    dc_.mixed(pf, dc)
+    pf2, dc2 = dc_.mixed_batches(3)
+    dc_.separate(pf2, dc2)
+    torch.cuda.synchronize()
+    assert torch.equal(pf["out"], pf2["out"]) and torch.equal(dc["out"], dc2["out"])
+    ref = oracle.attend(**case.oracle_kwargs())
+    n_pf = int(case.cu_q[3]) * hq
+    tol = edge_max_abs(case)
+    check(_f64(pf["out"]), ref[:n_pf], max_abs=tol, what="mixed: prefill part")
+    check(_f64(dc["out"]), ref[n_pf:], max_abs=tol, what="mixed: decode part")
+    assert dc_.status() == 0
+
+
+def test_mixed_step_orders_work_on_the_callers_stream():
+    """Work enqueued on the caller's stream after the call sees both outputs (the join), and the
+    side stream does not start before work enqueued before the call (the fork)."""
+    case = _mixed_case()
+    dc_ = DeviceCase(case)
+    pf, dc = dc_.mixed_batches(3)
+    ref_pf, ref_dc = dc_.mixed_batches(3)
+    dc_.separate(ref_pf, ref_dc)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        torch.cuda._sleep(2_000_000)         # the caller's stream is still busy at the fork ...
+        dc["out"].fill_(7.0)                 # ... with a write the decode must come after
+        dc_.mixed(pf, dc, stream=s)
+        got_dc = dc["out"].clone()           # after the call, on the caller's stream
+        got_pf = pf["out"].clone()
+    s.synchronize()
+    assert torch.equal(got_dc, ref_dc["out"]) and torch.equal(got_pf, ref_pf["out"])
+
+
+def test_mixed_step_in_a_cuda_graph():
+    case = _mixed_case()
+    dc_ = DeviceCase(case)
+    pf, dc = dc_.mixed_batches(3)
+    dc_.mixed(pf, dc)                        # first call on the device, outside the capture
+    torch.cuda.synchronize()
+    want_pf, want_dc = pf["out"].clone(), dc["out"].clone()
+    pf["out"].zero_()
+    dc["out"].zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        dc_.mixed(pf, dc)
+    for _ in range(2):
+        pf["out"].zero_()
+        dc["out"].zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(pf["out"], want_pf) and torch.equal(dc["out"], want_dc)
+    del g
+    assert dc_.status() == 0
+
+
 def test_queries_that_see_nothing_give_zero_rows():
     case = make_case(5, hq=8, hkv=2, d=128, requests=[([(0, 100, 20)], [50]), ([(20, 0, 16)], [15])])
     dc = DeviceCase(case)
