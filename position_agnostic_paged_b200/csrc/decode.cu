@@ -49,7 +49,7 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 // returns to the same warp: a warp's parity wait on a stage can then never
 // run ahead of that stage's previous round (which another warp would own).
 template <int NT, bool PLAIN, int kDecodeStages>
-__global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(kDecodeThreads, 3) decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                       const __grid_constant__ CUtensorMap tmV,
                                                                       const AttnParams p) {
     constexpr int KW = 4 / NT;   // warps sharing the words of one head group
@@ -93,39 +93,63 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
 
     if (warp == 4) {
         // ------------------------------------------------------------ producer
+        // The warp fetches the split's table words and their blocks' metadata 32 at a time,
+        // one word per lane (two dependent global loads per 32 words instead of per word);
+        // lane 0 then arms the stages in word order with the values shuffled to it.
         if (lane == 0) {
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            int issued = 0;
-            for (int i = 0; i < cnt; ++i) {
-                const int st = i % kDecodeStages;
-                const uint32_t ph = (i / kDecodeStages) & 1;
-                if (!mbar_wait(&empty_bar[st], ph ^ 1)) {
-                    set_status(p.d_status, LAZY_DSTATUS_TIMEOUT);
+        }
+        int issued = 0;
+        bool stop = false;
+        for (int i0 = 0; i0 < cnt && !stop; i0 += 32) {
+            uint32_t w_l = 0u, m_l = 0u;
+            if (i0 + lane < cnt) {
+                w_l = p.table[wbase + lo + i0 + lane];
+                const uint32_t b = word_block(w_l);
+                if (b < static_cast<uint32_t>(p.num_blocks)) m_l = p.blk_meta[b];
+            }
+            const int n = min(32, cnt - i0);
+            for (int k = 0; k < n; ++k) {
+                const uint32_t w = __shfl_sync(0xffffffffu, w_l, k);
+                const uint32_t meta = __shfl_sync(0xffffffffu, m_l, k);
+                if (lane == 0) {
+                    const int i = i0 + k;
+                    const int st = i % kDecodeStages;
+                    const uint32_t ph = (i / kDecodeStages) & 1;
+                    if (!mbar_wait(&empty_bar[st], ph ^ 1)) {
+                        set_status(p.d_status, LAZY_DSTATUS_TIMEOUT);
+                        stop = true;
+                    } else {
+                        const int widx = wbase + lo + i;
+                        const uint32_t b = word_block(w);
+                        issued = i + 1;
+                        // the word and the block's metadata travel with the stage, so
+                        // consumers read them from shared memory (the arrive releases them)
+                        stage_word[st] = w;
+                        if (b >= static_cast<uint32_t>(p.num_blocks)) {
+                            stage_meta[st] = 0u;
+                            set_status(p.d_status, LAZY_DSTATUS_BAD_BLOCK);
+                            mbar_arrive(&full_bar[st]);   // completes the phase with no data
+                        } else {
+                            stage_meta[st] = meta;
+                            mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
+                            uint8_t *dst = stages + st * kStageBytes;
+                            const int krow = PLAIN ? (widx * p.hkv + kvh) * kBlockTokens
+                                                   : (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens;
+                            const int vrow = (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens;
+                            tma_load_block(dst, &tmK, krow, &full_bar[st]);
+                            tma_load_block(dst + kBlockBytes, &tmV, vrow, &full_bar[st]);
+                        }
+                    }
+                }
+                if (__shfl_sync(0xffffffffu, stop ? 1 : 0, 0)) {
+                    stop = true;
                     break;
                 }
-                const int widx = wbase + lo + i;
-                const uint32_t w = p.table[widx];
-                const uint32_t b = word_block(w);
-                issued = i + 1;
-                // the word and the block's metadata travel with the stage, so
-                // consumers read them from shared memory (the arrive releases them)
-                stage_word[st] = w;
-                if (b >= static_cast<uint32_t>(p.num_blocks)) {
-                    stage_meta[st] = 0u;
-                    set_status(p.d_status, LAZY_DSTATUS_BAD_BLOCK);
-                    mbar_arrive(&full_bar[st]);   // completes the phase with no data
-                    continue;
-                }
-                stage_meta[st] = p.blk_meta[b];
-                mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
-                uint8_t *dst = stages + st * kStageBytes;
-                const int krow = PLAIN ? (widx * p.hkv + kvh) * kBlockTokens
-                                       : (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens;
-                const int vrow = (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens;
-                tma_load_block(dst, &tmK, krow, &full_bar[st]);
-                tma_load_block(dst + kBlockBytes, &tmV, vrow, &full_bar[st]);
             }
+        }
+        if (lane == 0) {
             // Never leave with copies in flight: wait for the last phase of
             // every stage this thread armed (immediate on the normal path).
             for (int i = max(0, issued - kDecodeStages); i < issued; ++i)
@@ -201,14 +225,16 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_split_kernel(const __gr
                 }
                 const uint32_t kbase = stage0 + st * kStageBytes;
                 const uint32_t vbase = kbase + kBlockBytes;
-                // S^T[16 keys][8 heads] = K q^T
-                float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+                // S^T[16 keys][8 heads] = K q^T, the 8 k-steps in two independent chains
+                float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sacc2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int s = 0; s < 8; ++s) {
                     uint32_t a0, a1, a2, a3;
                     ldsm_x4(kbase + swz_offset(k_key, 16 * s + k_dc, kBlockTokens), a0, a1, a2, a3);
-                    mma_bf16(sacc, a0, a1, a2, a3, qb[s][0], qb[s][1]);
+                    mma_bf16((s & 1) ? sacc2 : sacc, a0, a1, a2, a3, qb[s][0], qb[s][1]);
                 }
+#pragma unroll
+                for (int x = 0; x < 4; ++x) sacc[x] += sacc2[x];
                 const int j0 = meta_j0(meta), nv = meta_valid(meta);
                 if (p.alibi) {
                     // slope * (key position - query position) for keys rr and rr + 8
