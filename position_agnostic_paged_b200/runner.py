@@ -31,9 +31,10 @@ def cfg_of(wl: Workload) -> la.Cfg:
 
 
 class DevicePool:
-    def __init__(self, wl: Workload, device="cuda", sentinel: int | None = None):
+    def __init__(self, wl: Workload, device="cuda", sentinel: int | None = None, cfg: la.Cfg | None = None):
+        """cfg: the configuration every call on this pool uses (default: the workload's, RoPE)."""
         self.wl = wl
-        self.cfg = cfg_of(wl)
+        self.cfg = cfg_of(wl) if cfg is None else cfg
         self.device = torch.device(device)
         shape = (wl.num_blocks, wl.hkv, 16, wl.d)
         if sentinel is None:

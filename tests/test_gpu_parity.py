@@ -551,6 +551,59 @@ def test_prefill_8b_full_size():
     assert _run_full("prefill_8b", 64) == ["prefill"]
 
 
+@pytest.mark.parametrize("name", ["decode_8b", "prefill_8b"])
+def test_alibi_full_size(name):
+    """ALiBi at the benchmark's sizes and launch configuration: the pool written under ALiBi (keys
+    as given), sampled rows against the oracle."""
+    import dataclasses
+
+    from position_agnostic_paged_b200.runner import cfg_of
+    wl = W.make(name)
+    sp, so = _alibi_slopes(wl.hq)
+    pool = DevicePool(wl, cfg=dataclasses.replace(cfg_of(wl), alibi_slopes=tuple(sp))).setup()
+    step = wl.steps[0]
+    ds = DeviceStep(pool, step)
+    ds.write_new_tokens()
+    ds.attend()
+    torch.cuda.synchronize()
+    sq, sh = _sample_rows(step, wl.hq, 64, 9)
+    ref = oracle.attend(num_q_heads=wl.hq, num_kv_heads=wl.hkv, rope_base=wl.rope_base, q_raw=step.q_raw,
+                        cu_q=step.cu_q, q_pos=step.q_pos, seg_indptr=step.seg_indptr, seg_src=step.seg_src,
+                        seg_off=step.seg_off, seg_len=step.seg_len, k_tok=wl.k_store, v_tok=wl.v_store,
+                        sel_q=sq, sel_h=sh, alibi_slopes=so)
+    got = ds.out_f64().reshape(step.total_q, wl.hq, wl.d)
+    check(got[sq, sh], ref, what=f"{name} alibi sampled")
+    assert pool.status() == 0
+
+
+def test_mixed_step_full_size():
+    """lazy_mixed_attn on the mixed 8B step (32 prefill chunks + 192 decodes, 1 GiB pool): equal
+    bit for bit to the two separate calls, and sampled rows of both parts against the oracle."""
+    from position_agnostic_paged_b200.runner import mixed_attend
+    wl = W.make("mixed_8b")
+    pool = DevicePool(wl).setup()
+    by_kind = {st.kind: st for st in wl.steps}
+    pf, dc = DeviceStep(pool, by_kind["prefill"]), DeviceStep(pool, by_kind["decode"])
+    pf.write_new_tokens()
+    dc.write_new_tokens()
+    pf.attend()
+    dc.attend()
+    torch.cuda.synchronize()
+    want_pf, want_dc = pf.out.clone(), dc.out.clone()
+    pf.out.zero_()
+    dc.out.zero_()
+    mixed_attend(pf, dc)
+    torch.cuda.synchronize()
+    assert torch.equal(pf.out, want_pf) and torch.equal(dc.out, want_dc)
+    for ds in (pf, dc):
+        st = ds.step
+        sq, sh = _sample_rows(st, wl.hq, 32, 11)
+        ref = oracle_step(wl, st, sq, sh)
+        got = ds.out_f64().reshape(st.total_q, wl.hq, wl.d)
+        check(got[sq, sh], ref, what=f"mixed step {st.kind} sampled")
+    assert pool.status() == 0
+
+
 @pytest.mark.slow
 def test_decode_70b_full_size():
     assert _run_full("decode_70b", 24) == ["decode"]
