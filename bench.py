@@ -165,26 +165,35 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(world, x: float) -> float:
+def _all_reduce(world, x: float, op_name: str) -> float:
+    """x reduced over the ranks (timings and counts only; the path itself exchanges nothing).
+    The tensor lives where the process group's backend wants it: the GPU for NCCL, the host for
+    gloo (the multi-rank logic is tested on CPU with gloo)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=getattr(dist.ReduceOp, op_name))
     return float(t.item())
+
+
+def max_over_ranks(world, x: float) -> float:
+    return _all_reduce(world, x, "MAX")
 
 
 def sum_over_ranks(world, x: float) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
+    return _all_reduce(world, x, "SUM")
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+
+def whole_job(world, local_units: float, local_ms: float):
+    """Whole-job throughput of independent replicas: the units all ranks processed divided by the
+    slowest rank's time.  Returns (units per second, that time in ms)."""
+    ms = max_over_ranks(world, local_ms)
+    units = sum_over_ranks(world, float(local_units))
+    return units / (ms * 1e-3), ms
 
 
 # ----------------------------------------------------------------------------- timing helpers
@@ -267,10 +276,9 @@ def run_ours(args):
     clocks.start()
     total_ms, attn_ms = timed_steps(decode_step, args.steps, args.warmup, flush, world, inner=True)
     clk = clocks.stop()
-    ms_step = max_over_ranks(world, total_ms / args.steps)
+    rate, ms_step = whole_job(world, dec_bytes, total_ms / args.steps)
     attn_avg = max_over_ranks(world, float(np.mean(attn_ms)))
-    all_bytes = sum_over_ranks(world, float(dec_bytes))
-    value = all_bytes / (ms_step * 1e-3) / 1e9
+    value = rate / 1e9
     achieved = dec_bytes / (attn_avg * 1e-3) / 1e9
     if pool.status() != 0:
         raise SystemExit(f"device status {pool.status()} after decode steps")
@@ -410,9 +418,8 @@ def run_e2e(ds, pool, step, dec_bytes, args, world):
         out_h.copy_(ds.out.view(torch.int16), non_blocking=True)
 
     total, _ = timed_steps(e2e_step, args.steps, args.warmup, flush, world)
-    ms = max_over_ranks(world, total / args.steps)
-    all_bytes = sum_over_ranks(world, float(dec_bytes))
-    return {"value": round(all_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 5),
+    rate, ms = whole_job(world, dec_bytes, total / args.steps)
+    return {"value": round(rate / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 5),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
@@ -456,11 +463,10 @@ def run_prefill(args, world, peaks, peak_src, flush):
             ev[1].record()
 
     total, attn = timed_steps(pf_step, args.steps, args.warmup, flush, world, inner=True)
-    ms = max_over_ranks(world, total / args.steps)
+    rate, ms = whole_job(world, flops, total / args.steps)
     attn_avg = max_over_ranks(world, float(np.mean(attn)))
     if pool.status() != 0:
         raise SystemExit(f"device status {pool.status()} after prefill steps")
-    all_flops = sum_over_ranks(world, float(flops))
     achieved = flops / (attn_avg * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     comparison = None
@@ -496,7 +502,7 @@ def run_prefill(args, world, peaks, peak_src, flush):
         "_launches": launches,
         "workload": "prefill_8b: Llama-3.1-8B shapes, 16 requests x 256 causal query tokens over 10 Zipf(1.0) "
                     "docs x 512 (5376 keys), 1000-doc pool",
-        "value": round(all_flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
+        "value": round(rate / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 5),
         "step": "lazy_kv_write(256-token chunks) + lazy_prefill_attn",
         "algorithmic_flops_per_launch": flops,
         "roofline": {"bound": "tensor", "kernel": "lazy_prefill_attn", "achieved": round(achieved, 1),
