@@ -54,7 +54,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TRAFFIC = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
     #     -k regex:decode_split -s 3 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu --no-compare --no-e2e
-    "decode_8b": {"sha": "3cb8abcea00ce0df", "bytes": 785442560 + 6835200},
+    "decode_8b": {"sha": "0124832b79ae54bb", "bytes": 785284352 + 8163072},
     # the same with -k regex:prefill_tc
     "prefill_8b": {"sha": "e766bd345ac84128", "bytes": 300506624 + 25670912},
 }

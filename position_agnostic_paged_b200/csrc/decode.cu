@@ -260,7 +260,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_split_kernel(const _
                 for (int j = 0; j < 2; ++j) {
                     const float mn = fmaxf(m_run[j], bm[j]);
                     const float mu = mn == -INFINITY ? 0.f : mn;
-                    const float sc = fast_exp2(m_run[j] - mu);
+                    // the rescale factor is exactly 1 while the running max stands (most words)
+                    float sc = 1.f;
+                    if (mn != m_run[j]) sc = fast_exp2(m_run[j] - mu);
                     if (sc != 1.f) {
                         l_run[j] *= sc;
 #pragma unroll
