@@ -128,6 +128,29 @@ __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v 
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 __device__ __forceinline__ float bits_to_float(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
 
+// Paired fp32 arithmetic (sm_100: one instruction for two lanes of work, each
+// element rounded exactly as the scalar operation would round it).
+// (a0, a1) += (b0, b1)
+__device__ __forceinline__ void add2(float &a0, float &a1, float b0, float b1) {
+    asm("{\n .reg .b64 x, y;\n mov.b64 x, {%0, %1};\n mov.b64 y, {%2, %3};\n add.rn.f32x2 x, x, y;\n"
+        " mov.b64 {%0, %1}, x;\n}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(b0), "f"(b1));
+}
+// (a0, a1) = (m * b0 + a0, m * b1 + a1)
+__device__ __forceinline__ void fma2(float &a0, float &a1, float m, float b0, float b1) {
+    asm("{\n .reg .b64 x, y, z;\n mov.b64 x, {%0, %1};\n mov.b64 y, {%2, %2};\n mov.b64 z, {%3, %4};\n"
+        " fma.rn.f32x2 x, y, z, x;\n mov.b64 {%0, %1}, x;\n}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(m), "f"(b0), "f"(b1));
+}
+// max(a, b, c) in one instruction (exact)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // 2^x via the SFU (PTX ex2.approx, relative error about 2^-22); 2^-inf = 0.
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;

@@ -526,35 +526,40 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 // the in-block part of the bias, slope * s for slot s; the block part bk[k] enters
                 // the block maxima and the exponent's offset below (one op per score, not two)
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    sv[c] = __float_as_uint(fmaf(slope, static_cast<float>(c & 15), __uint_as_float(sv[c])));
+                for (int c = 0; c < 128; c += 2) {
+                    float x0 = __uint_as_float(sv[c]), x1 = __uint_as_float(sv[c + 1]);
+                    fma2(x0, x1, slope, static_cast<float>(c & 15), static_cast<float>((c + 1) & 15));
+                    sv[c] = __float_as_uint(x0);
+                    sv[c + 1] = __float_as_uint(x1);
+                }
             }
             if (!full) {
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
                     sv[c] = (c & 15) < lim[c >> 4] ? sv[c] : 0xFF800000u;   // -inf: P = 0
             }
-            float m0 = __uint_as_float(sv[0]), m1 = __uint_as_float(sv[1]);
+            // row max with three-input maxima (exact, so the order does not matter)
+            auto f = [&](int c) { return __uint_as_float(sv[c]); };
+            float m0 = f(0), m1 = f(1);
             if (ALIBI) {
                 // row max of (score + bias): per 16-key block, the block part added once
                 m0 = -INFINITY;
 #pragma unroll
                 for (int k = 0; k < kTileBlocks; ++k) {
-                    float a = __uint_as_float(sv[16 * k]), b = __uint_as_float(sv[16 * k + 1]);
+                    float a = max3(f(16 * k), f(16 * k + 1), f(16 * k + 2));
 #pragma unroll
-                    for (int c = 2; c < 16; c += 2) {
-                        a = fmaxf(a, __uint_as_float(sv[16 * k + c]));
-                        b = fmaxf(b, __uint_as_float(sv[16 * k + c + 1]));
-                    }
-                    m0 = fmaxf(m0, fmaxf(a, b) + bk[k]);
+                    for (int c = 3; c < 15; c += 2) a = max3(a, f(16 * k + c), f(16 * k + c + 1));
+                    a = fmaxf(a, f(16 * k + 15));
+                    m0 = fmaxf(m0, a + bk[k]);
                 }
                 m1 = m0;
             } else {
 #pragma unroll
-                for (int c = 2; c < 128; c += 2) {
-                    m0 = fmaxf(m0, __uint_as_float(sv[c]));
-                    m1 = fmaxf(m1, __uint_as_float(sv[c + 1]));
+                for (int c = 2; c < 126; c += 4) {
+                    m0 = max3(m0, f(c), f(c + 1));
+                    m1 = max3(m1, f(c + 2), f(c + 3));
                 }
+                m0 = max3(m0, f(126), f(127));
             }
             const float m_new = fmaxf(m_run, fmaxf(m0, m1));
             const bool need = m_new > m_run + kRescaleThreshold;
@@ -570,15 +575,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
                 for (int k = 0; k < kTileBlocks; ++k) bk[k] = mu - bk[k];
             }
-            // P = 2^(S - m) as bf16 pairs over the first 64 columns of S, row sum in fp32
+            // P = 2^(S - m) as bf16 pairs over the first 64 columns of S, row sums (even and
+            // odd columns) in fp32; the subtraction and the sums run as paired fp32 operations
             float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
             for (int e = 0; e < 64; ++e) {
-                const float mo = ALIBI ? bk[e >> 3] : mu;
-                const float p0 = fast_exp2(__uint_as_float(sv[2 * e]) - mo);
-                const float p1 = fast_exp2(__uint_as_float(sv[2 * e + 1]) - mo);
-                ls0 += p0;
-                ls1 += p1;
+                const float nmo = -(ALIBI ? bk[e >> 3] : mu);
+                float x0 = f(2 * e), x1 = f(2 * e + 1);
+                add2(x0, x1, nmo, nmo);
+                const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                add2(ls0, ls1, p0, p1);
                 sv[e] = pack_bf16(p0, p1);
             }
             tc::st32(tS + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(sv + 0));
