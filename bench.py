@@ -56,7 +56,7 @@ TRAFFIC = {
     #     -k regex:decode_split -s 3 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu --no-compare --no-e2e
     "decode_8b": {"sha": "0124832b79ae54bb", "bytes": 785284352 + 8163072},
     # the same with -k regex:prefill_tc
-    "prefill_8b": {"sha": "1c713efe94807cce", "bytes": 302907648 + 27202816},
+    "prefill_8b": {"sha": "540713ca02456b05", "bytes": 303353600 + 26622720},
 }
 
 

@@ -144,6 +144,21 @@ __device__ __forceinline__ void fma2(float &a0, float &a1, float m, float b0, fl
         : "+f"(a0), "+f"(a1)
         : "f"(m), "f"(b0), "f"(b1));
 }
+// (x0, x1) = (p0 * q0 + a0, p1 * q1 + a1)
+__device__ __forceinline__ void fma2v(float &x0, float &x1, float p0, float p1, float q0, float q1, float a0,
+                                      float a1) {
+    asm("{\n .reg .b64 p, q, a;\n mov.b64 p, {%2, %3};\n mov.b64 q, {%4, %5};\n mov.b64 a, {%6, %7};\n"
+        " fma.rn.f32x2 p, p, q, a;\n mov.b64 {%0, %1}, p;\n}"
+        : "=f"(x0), "=f"(x1)
+        : "f"(p0), "f"(p1), "f"(q0), "f"(q1), "f"(a0), "f"(a1));
+}
+// (x0, x1) = (p0 * q0, p1 * q1)
+__device__ __forceinline__ void mul2(float &x0, float &x1, float p0, float p1, float q0, float q1) {
+    asm("{\n .reg .b64 p, q;\n mov.b64 p, {%2, %3};\n mov.b64 q, {%4, %5};\n mul.rn.f32x2 p, p, q;\n"
+        " mov.b64 {%0, %1}, p;\n}"
+        : "=f"(x0), "=f"(x1)
+        : "f"(p0), "f"(p1), "f"(q0), "f"(q1));
+}
 // max(a, b, c) in one instruction (exact)
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;

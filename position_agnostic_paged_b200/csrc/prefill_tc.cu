@@ -704,11 +704,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                         uint32_t *hw = reinterpret_cast<uint32_t *>(&hi);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
+                            // (a, b) -> (a c - b s, b c + a s) for two pairs at once (paired fp32)
                             const float a0 = bf16_lo(aw[e]), a1 = bf16_hi(aw[e]);
                             const float b0 = bf16_lo(bw[e]), b1 = bf16_hi(bw[e]);
                             const float c0 = kc[2 * e], s0 = kn[2 * e], c1 = kc[2 * e + 1], s1 = kn[2 * e + 1];
-                            lw[e] = pack_bf16(a0 * c0 - b0 * s0, a1 * c1 - b1 * s1);
-                            hw[e] = pack_bf16(b0 * c0 + a0 * s0, b1 * c1 + a1 * s1);
+                            float ac0, ac1, bc0, bc1, lo0, lo1, hi0, hi1;
+                            mul2(ac0, ac1, a0, a1, c0, c1);
+                            mul2(bc0, bc1, b0, b1, c0, c1);
+                            fma2v(lo0, lo1, -b0, -b1, s0, s1, ac0, ac1);
+                            fma2v(hi0, hi1, a0, a1, s0, s1, bc0, bc1);
+                            lw[e] = pack_bf16(lo0, lo1);
+                            hw[e] = pack_bf16(hi0, hi1);
                         }
                         *reinterpret_cast<uint4 *>(kt + soff) = lo;
                         *reinterpret_cast<uint4 *>(kt + kHalfPlane + soff) = hi;
