@@ -1,7 +1,8 @@
 """Benchmark of the deferred-RoPE paged attention hot path on B200.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                [--workload decode_8b] [--no-prefill] [--no-compare] [--no-e2e]
+                [--workload decode_8b] [--no-prefill] [--no-compare] [--no-e2e] [--no-cpu]
+                [--extended] [--cache-sim] [--profile-case NAME]
 
 One step (ours) = one pass of the hot path over one batch of the decode
 workload with Llama-3.1-8B attention shapes (64 requests, 32/8 heads, d 128,
@@ -16,9 +17,10 @@ a 512 MiB buffer outside the timed intervals.
 Also measured in the same run and reported in sub-objects:
   prefill     the causal prefill workload with 8B shapes (16 requests x 256
               query tokens over 10 documents), TFLOP/s over visible pairs;
-  comparison  the position-aware alternative on the same inputs (and the same attention with ALiBi
-              in place of RoPE, timing only):
-              materialise re-rotated keys, then plain paged attention;
+  comparison  the position-aware alternative on the same inputs: materialise
+              re-rotated keys, then plain paged attention; also the rotation-off
+              kernel, and the same attention with ALiBi in place of RoPE (timing
+              only);
   e2e         the decode metric through the same C-ABI calls with the step's
               inputs copied from pinned host memory and the output copied back
               inside the timed region;
@@ -27,7 +29,14 @@ Also measured in the same run and reported in sub-objects:
 --impl reference times the fp64 CPU oracle itself (the only reference
 implementation this project has) on a bounded sample of the same workload.
 Multi-GPU: one independent replica per rank (the path needs no exchange step);
-the time is the maximum over ranks.
+the time is the maximum over ranks and the work the sum over ranks.
+
+--extended adds decode at 70B shapes (Zipf 1.2 and uniform popularity) and the
+mixed 8B serving step (GQA and MQA), with the whole step timed as two calls
+and as one lazy_mixed_attn call.  --cache-sim runs the host-side cache-hit
+simulation of position-agnostic, position-aware and prefix caching (no GPU).
+--profile-case launches only the attention kernel of a small case, for
+profiler captures.
 """
 from __future__ import annotations
 
