@@ -106,3 +106,20 @@ def compare(budget_bytes: float = 2 ** 30, alphas=(0.6, 1.0, 1.4), seed: int = 1
         rows.append({"alpha": a, "budget_bytes": int(budget_bytes), "capacity_blocks": cap,
                      **{f"hit_ratio_{k}": round(v, 4) for k, v in res.items()}, **gain})
     return rows
+
+
+def budget_sweep(budgets_gb=(0.125, 0.25, 0.5, 1, 2, 4, 8), alpha: float = 1.0, seed: int = 1005,
+                 n_requests: int = 6000, **stream_kw) -> list[dict]:
+    """Hit ratios of the policies across KV budgets at one Zipf exponent: how the gains of
+    position-agnostic caching move with the pressure on the budget."""
+    from .workloads import cache_stream
+    lens, reqs = cache_stream(seed, alpha=alpha, n_requests=n_requests, **stream_kw)
+    rows = []
+    for gb in budgets_gb:
+        cap = int(gb * 2 ** 30 // kv_bytes_per_block())
+        res = {pol: simulate(pol, lens, reqs, cap)["hit_ratio"] for pol in POLICIES}
+        gain = {f"gain_vs_{k}": round(res["agnostic"] / res[k], 2) if res[k] else None for k in POLICIES[1:]}
+        rows.append({"alpha": alpha, "budget_bytes": int(gb * 2 ** 30), "capacity_blocks": cap,
+                     **{f"hit_ratio_{k}": round(v, 4) for k, v in res.items()}, **gain})
+    return rows
+

@@ -190,3 +190,14 @@ def test_cache_stream_shape_and_skew():
     counts = np.bincount(reqs.ravel(), minlength=500)
     top = np.sort(counts)[::-1]
     assert top[:10].sum() > 5 * top[250:260].sum()       # skewed popularity
+
+
+def test_budget_sweep_rows():
+    rows = cache_sim.budget_sweep(budgets_gb=(0.25, 1), n_requests=150, n_docs=300)
+    assert [r["capacity_blocks"] for r in rows] == [int(g * 2 ** 30 // cache_sim.kv_bytes_per_block())
+                                                  for g in (0.25, 1)]
+    for r in rows:
+        for p in cache_sim.POLICIES:
+            assert 0.0 <= r[f"hit_ratio_{p}"] <= 1.0
+        # one copy per document never loses to keying copies by offset or by sequence here
+        assert r["hit_ratio_agnostic"] >= max(r["hit_ratio_aware"], r["hit_ratio_aware_exact"], r["hit_ratio_prefix"])
