@@ -128,3 +128,13 @@ def test_mixed_step_validates_both_batches_before_launching():
     assert call(c, None, None) == la.LAZY_OK              # nothing to do
     bad_pf = la.PrefillBatch(1, 1, 1, 2, -1, 4, 1, 1, 4, 1, 1, 1 << 20)
     assert call(c, bad_pf, la.DecodeBatch(1, 1, 2, 1, 1, 4, 1, 3, 1 << 20)) == la.LAZY_EINVAL
+
+
+def test_position_tables_agree_with_the_oracle_s_own():
+    """The library's RoPE-variant and ALiBi tables and the oracle's are two independent
+    computations of the published rules; they must agree."""
+    from position_agnostic_paged_b200 import rope
+    np.testing.assert_allclose(rope.llama31_theta(), oracle.llama31_theta(), rtol=1e-14, atol=0)
+    np.testing.assert_allclose(rope.default_theta(), 500000.0 ** (-(2.0 * np.arange(64)) / 128), rtol=1e-15)
+    for n in (1, 2, 3, 5, 6, 8, 12, 16, 24, 32, 40, 64, 96, 128):
+        np.testing.assert_allclose(rope.alibi_slopes(n), oracle.alibi_slopes(n), rtol=1e-14, atol=0)
