@@ -60,12 +60,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch of the dominant kernels from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the SHA-256 of the
 # kernel source it was taken on; reported as null when the source changed.
+# Each figure holds for the kernel source whose hash it carries; a source edit voids it, except an
+# edit of comments alone (same lines), after which the hash is re-pinned.
 TRAFFIC = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
     #     -k regex:decode_split -s 3 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu --no-compare --no-e2e
-    "decode_8b": {"sha": "0124832b79ae54bb", "bytes": 785284352 + 8163072},
+    "decode_8b": {"sha": "c5296f2fb7ad0da4", "bytes": 785284352 + 8163072},
     # the same with -k regex:prefill_tc
-    "prefill_8b": {"sha": "540713ca02456b05", "bytes": 303353600 + 26622720},
+    "prefill_8b": {"sha": "a67e527ec670daa8", "bytes": 303353600 + 26622720},
 }
 
 

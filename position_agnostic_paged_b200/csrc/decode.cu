@@ -3,8 +3,8 @@
 // Source: gist.science, "LazyAttention: Efficient Retrieval-Augmented
 // Generation with Deferred Positional Encoding", Technical Summary, Technical
 // Implementation: Decoding -- one query token per request (M = 1); the
-// rotation is fused into the inner loop and the query is rotated only when
-// the relative offset changes (a new document); the (block ID, offset)
+// rotation lives inside the inner loop, and the query is rotated again just
+// at a change of segment offset (a new document); the (block ID, offset)
 // metadata is decoded from one register; the kernel reads only K and V.
 //
 // Work decomposition.  One CTA per (split, KV head, request); a split is a

@@ -4,10 +4,10 @@
 //
 // Source: gist.science, "LazyAttention: Efficient Retrieval-Augmented
 // Generation with Deferred Positional Encoding", Technical Summary, Technical
-// Implementation: Prefilling -- the kernel loads cached KV blocks and applies
-// one relative rotation based on the offset between the query and the cached
-// document instead of resetting the keys to position 0 and rotating them
-// again; this phase is compute-bound.
+// Implementation: Prefilling -- the kernel reads the cached KV blocks and
+// rotates once, by the distance from the cached document's offset to the
+// query's position, rather than taking the keys back to position 0 and
+// rotating them a second time; this phase is bound by compute.
 //
 // Where the single relative rotation goes.  Keys sit in the pool rotated at
 // their local index j.  Each CTA fixes a reference position P0 (its first
