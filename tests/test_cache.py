@@ -201,3 +201,15 @@ def test_budget_sweep_rows():
             assert 0.0 <= r[f"hit_ratio_{p}"] <= 1.0
         # one copy per document never loses to keying copies by offset or by sequence here
         assert r["hit_ratio_agnostic"] >= max(r["hit_ratio_aware"], r["hit_ratio_aware_exact"], r["hit_ratio_prefix"])
+
+
+def test_cache_capacity_is_bounded_by_the_block_id_field():
+    # block ids are 17 bits in the table word, so a cache over more blocks cannot be addressed
+    c = BlockCache(1 << 17)
+    try:
+        hit, blocks = c.access(1, 5)
+        assert not hit and blocks.tolist() == [0, 1, 2, 3, 4]
+    finally:
+        c.close()
+    with pytest.raises(Exception):
+        BlockCache((1 << 17) + 1)
