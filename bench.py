@@ -693,14 +693,18 @@ def run_profile_case(args):
 def run_cache_sim(args):
     """Cache-hit ratios of position-agnostic caching against position-aware (re-encoding and
     exact-offset) and prefix caching, at a 1 GB KV budget of Llama-3.1-8B geometry, for three Zipf
-    exponents of document popularity, then across budgets from 128 MB to 8 GB at Zipf 1.0; host
-    only, one JSON line per exponent or budget."""
+    exponents of document popularity (documents in random order, then ordered by popularity rank),
+    then across budgets from 128 MB to 8 GB at Zipf 1.0; host only, one JSON line per exponent or
+    budget."""
     from position_agnostic_paged_b200 import cache_sim
     t0 = time.perf_counter()
+    n_sweep = max(1, args.cache_requests * 3 // 10)
     for row in cache_sim.compare(n_requests=args.cache_requests):
         print(json.dumps({"metric": "cache_hit_ratio", "unit": "fraction of document blocks",
                           "data": "synthetic", "requests": args.cache_requests, **row}), flush=True)
-    n_sweep = max(1, args.cache_requests * 3 // 10)
+    for row in cache_sim.compare(n_requests=n_sweep, order="rank"):
+        print(json.dumps({"metric": "cache_hit_ratio", "unit": "fraction of document blocks",
+                          "data": "synthetic", "requests": n_sweep, **row}), flush=True)
     for row in cache_sim.budget_sweep(n_requests=n_sweep):
         print(json.dumps({"metric": "cache_hit_ratio", "unit": "fraction of document blocks",
                           "data": "synthetic", "requests": n_sweep, "sweep": "budget", **row}), flush=True)

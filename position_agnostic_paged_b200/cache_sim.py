@@ -93,17 +93,17 @@ def kv_bytes_per_block(num_kv_heads: int = 8, head_dim: int = 128, block_tokens:
 
 
 def compare(budget_bytes: float = 2 ** 30, alphas=(0.6, 1.0, 1.4), seed: int = 1005, n_requests: int = 20000,
-            **stream_kw) -> list[dict]:
+            order: str = "random", **stream_kw) -> list[dict]:
     """Hit ratios of the three policies per Zipf exponent at one KV budget (Llama-3.1-8B KV
     geometry: 8 KV heads x 128, bf16), with the gains of position-agnostic caching."""
     from .workloads import cache_stream
     cap = int(budget_bytes // kv_bytes_per_block())
     rows = []
     for a in alphas:
-        lens, reqs = cache_stream(seed, alpha=a, n_requests=n_requests, **stream_kw)
+        lens, reqs = cache_stream(seed, alpha=a, n_requests=n_requests, order=order, **stream_kw)
         res = {pol: simulate(pol, lens, reqs, cap)["hit_ratio"] for pol in POLICIES}
         gain = {f"gain_vs_{k}": round(res["agnostic"] / res[k], 2) if res[k] else None for k in POLICIES[1:]}
-        rows.append({"alpha": a, "budget_bytes": int(budget_bytes), "capacity_blocks": cap,
+        rows.append({"alpha": a, "order": order, "budget_bytes": int(budget_bytes), "capacity_blocks": cap,
                      **{f"hit_ratio_{k}": round(v, 4) for k, v in res.items()}, **gain})
     return rows
 

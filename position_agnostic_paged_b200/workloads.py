@@ -387,10 +387,14 @@ def with_overrides(step: Step, **kw) -> Step:
 
 # ----------------------------------------------------------------------------- cache-hit streams
 def cache_stream(seed: int, n_docs: int = 4000, doc_len=(128, 2048), docs_per_req: int = 8,
-                 alpha: float = 1.0, n_requests: int = 20000):
+                 alpha: float = 1.0, n_requests: int = 20000, order: str = "random"):
     """A seeded stream of RAG requests for cache simulations: per request, docs_per_req distinct
-    documents drawn from a finite Zipf(alpha) popularity (rank k has weight k^-alpha), in random
-    order.  Returns (doc_tokens [n_docs] int64, requests [n_requests][docs_per_req] int64)."""
+    documents drawn from a finite Zipf(alpha) popularity (rank k has weight k^-alpha), placed in
+    random order (order="random") or by popularity rank, most popular first (order="rank", a
+    stand-in for ordering by retrieval score).  Returns (doc_tokens [n_docs] int64,
+    requests [n_requests][docs_per_req] int64)."""
+    if order not in ("random", "rank"):
+        raise ValueError(order)
     rng = np.random.default_rng(seed)
     lens = rng.integers(doc_len[0], doc_len[1] + 1, n_docs).astype(np.int64)
     pop = rng.permutation(n_docs)             # document id of popularity rank k
@@ -398,6 +402,9 @@ def cache_stream(seed: int, n_docs: int = 4000, doc_len=(128, 2048), docs_per_re
     reqs = np.empty((n_requests, docs_per_req), np.int64)
     for r in range(n_requests):
         ranks = rng.choice(n_docs, size=docs_per_req, replace=False, p=w)
+        if order == "rank":
+            ranks = np.sort(ranks)
         reqs[r] = pop[ranks]
-        rng.shuffle(reqs[r])
+        if order == "random":
+            rng.shuffle(reqs[r])
     return lens, reqs

@@ -213,3 +213,14 @@ def test_cache_capacity_is_bounded_by_the_block_id_field():
         c.close()
     with pytest.raises(Exception):
         BlockCache((1 << 17) + 1)
+
+
+def test_cache_stream_rank_order():
+    lens, ranked = cache_stream(3, n_docs=500, docs_per_req=6, alpha=1.2, n_requests=1500, order="rank")
+    counts = np.bincount(ranked.ravel(), minlength=500)
+    top = int(np.argmax(counts))
+    # the most popular document, whenever drawn, comes first
+    rows = np.flatnonzero((ranked == top).any(axis=1))
+    assert rows.size > 100 and np.all(ranked[rows, 0] == top)
+    with pytest.raises(ValueError):
+        cache_stream(3, n_requests=2, order="sorted")
