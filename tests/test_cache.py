@@ -224,3 +224,33 @@ def test_cache_stream_rank_order():
     assert rows.size > 100 and np.all(ranked[rows, 0] == top)
     with pytest.raises(ValueError):
         cache_stream(3, n_requests=2, order="sorted")
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=60, deadline=None)
+@given(cap=st.integers(1, 40),
+       ops=st.lists(st.tuples(st.integers(0, 15), st.integers(1, 45)), min_size=1, max_size=120))
+def test_native_cache_matches_reference_on_arbitrary_sequences(cap, ops):
+    """Any sequence of (key, size) uses: the same hits as the reference LRU, and after every use
+    the cached entries' blocks are disjoint, in range and add up to the blocks in use."""
+    sizes = {}
+    ref, nat, held = RefLRU(cap), BlockCache(cap), {}
+    try:
+        for key, n in ops:
+            n = sizes.setdefault(key, n)            # an entry keeps its size
+            want = ref.access(key, n)
+            got, blocks = nat.access(key, n)
+            assert got is want
+            if blocks is not None:
+                held[key] = blocks
+            live = [held[k] for k in ref.entries]
+            allb = np.concatenate(live) if live else np.zeros(0, np.int32)
+            assert len(set(allb.tolist())) == allb.size == ref.used
+            assert allb.size == 0 or (allb.min() >= 0 and allb.max() < cap)
+        st_ = nat.stats()
+        assert st_["used_blocks"] == ref.used and st_["entries"] == len(ref.entries)
+        assert st_["evictions"] == ref.evictions
+    finally:
+        nat.close()
