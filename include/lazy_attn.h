@@ -21,7 +21,8 @@
  *   - Ownership: the caller allocates and frees every buffer (pools, tables,
  *     outputs, workspaces).  The library allocates no device memory and keeps
  *     no state between calls, except the fixed scratch array that
- *     lazy_decode_attn_noalloc uses (described at its declaration).
+ *     lazy_decode_attn_noalloc uses and the per-device side stream of
+ *     lazy_mixed_attn (each described at its declaration).
  *   - Errors found on the host (bad shapes, null pointers, a workspace too
  *     small) are returned BEFORE anything is launched.  A launch failure
  *     returns LAZY_ECUDA.
@@ -203,8 +204,14 @@ size_t lazy_prefill_workspace_bytes(const lazy_attn_cfg *cfg, int num_req, int t
  * q_raw: bf16 [total_q][Hq][128]; request r owns tokens cu_q[r] .. cu_q[r+1]-1
  * at positions q_pos0[r] + i.  max_q: host upper bound of tokens per request;
  * max_words as for decode.  out: bf16 [total_q][Hq][128].
- * For each segment the query tile is rotated once by (p_i - offset): one
- * relative rotation, not a reset to position 0 and a re-rotation. */
+ * Each CTA (256 query rows of one KV head) rotates its query rows once by
+ * (p_i - P0), P0 its first query position, and every key tile once by
+ * (o - P0), o the tile's segment offset: one relative rotation per tile, not
+ * a reset to position 0 and a re-rotation; scores carry (p_i - o - j).
+ * Tensor cores (tcgen05, accumulators in tensor memory); with the workspace
+ * of lazy_prefill_workspace_bytes, a second kernel merges split units.
+ * Under ALiBi (cfg.alibi_slopes) nothing is rotated and the bias is added to
+ * the scores instead. */
 int lazy_prefill_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *cu_q,
                       const int32_t *q_pos0, int num_req, int total_q, int max_q,
                       const uint32_t *table, const int32_t *table_indptr, int max_words,
