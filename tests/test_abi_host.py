@@ -138,3 +138,27 @@ def test_position_tables_agree_with_the_oracle_s_own():
     np.testing.assert_allclose(rope.default_theta(), 500000.0 ** (-(2.0 * np.arange(64)) / 128), rtol=1e-15)
     for n in (1, 2, 3, 5, 6, 8, 12, 16, 24, 32, 40, 64, 96, 128):
         np.testing.assert_allclose(rope.alibi_slopes(n), oracle.alibi_slopes(n), rtol=1e-14, atol=0)
+
+
+def test_header_is_plain_c_and_cxx(tmp_path):
+    """The public header compiles as C99 and C++11 on its own, and its inline codec packs words as
+    documented (a C program built against the header alone, no CUDA)."""
+    import shutil
+    import subprocess
+    inc = os.path.dirname(HEADER)
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    for lang, std in (("c", "-std=c99"), ("c++", "-std=c++11")):
+        cc = "gcc" if lang == "c" else "g++"
+        r = subprocess.run([cc, "-x", lang, std, "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-I", inc, HEADER],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+    src = tmp_path / "t.c"
+    src.write_text('#include "lazy_attn.h"\n'
+                   'int main(void) {\n'
+                   '  uint32_t w = lazy_pack(131071u, 32767u);\n'
+                   '  return (lazy_block(w) == 131071u && lazy_offset(w) == 32767u && lazy_pack(5u, 100u) == '
+                   '((100u << 17) | 5u)) ? 0 : 1;\n}\n')
+    exe = tmp_path / "t"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", inc, str(src), "-o", str(exe)], check=True)
+    assert subprocess.run([str(exe)]).returncode == 0
