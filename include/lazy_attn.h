@@ -333,6 +333,37 @@ int lazy_cache_contains(const lazy_block_cache *cache, uint64_t key);
  * cached entries, free extents. */
 int lazy_cache_stats(const lazy_block_cache *cache, int64_t *stats);
 
+/* ---- position-encoding tables (host) ----
+ * Tables for lazy_attn_cfg.rope_theta and lazy_attn_cfg.alibi_slopes ([CON]:
+ * the deferred encoding carries over to other relative encodings, RoPE
+ * variants and ALiBi; the pages fix no table, so each function follows the
+ * published rule it names).  All pointers are HOST pointers to caller-owned
+ * arrays; nothing is launched.  Each returns LAZY_OK, or LAZY_EINVAL (and
+ * writes nothing) for a null pointer or an argument outside its domain. */
+
+/* theta[i] = base^(-2i/head_dim), i < head_dim/2 (head_dim even, base > 1):
+ * the table the kernels use when rope_theta is NULL. */
+int lazy_rope_theta(double base, int head_dim, double *theta);
+
+/* Llama-3.1 frequency scaling (the "llama3" rope type of the Llama 3.1 model
+ * configuration; Llama 3.1 itself uses base 500000, factor 8, low 1, high 4,
+ * original context 8192).  With f_i = base^(-2i/head_dim) and wavelength
+ * 2 pi / f_i: wavelengths below original_max_position / high_freq_factor keep
+ * f_i, those above original_max_position / low_freq_factor get f_i / factor,
+ * and in between theta_i = t f_i + (1 - t) f_i / factor with
+ * t = (original_max_position / wavelength - low) / (high - low).
+ * Needs factor > 0, 0 < low_freq_factor < high_freq_factor,
+ * original_max_position > 0.  theta: head_dim/2 doubles. */
+int lazy_rope_theta_llama31(double base, int head_dim, double factor, double low_freq_factor,
+                            double high_freq_factor, double original_max_position, double *theta);
+
+/* ALiBi head slopes (Press, Smith and Lewis, "Train Short, Test Long", 2022):
+ * for a power of two n, slope k = 2^(-8k/n), k = 1..n; otherwise the slopes
+ * of the largest power of two p below num_heads, then every second slope
+ * (1st, 3rd, ...) of the 2p-head rule, num_heads - p of them.
+ * slopes: num_heads doubles (num_heads >= 1). */
+int lazy_alibi_slopes(int num_heads, double *slopes);
+
 /* ---- test export ---- */
 
 /* Decodes n_words table words on the device, exactly as the attention kernels

@@ -27,7 +27,7 @@ EXPORTED = [
     "lazy_materialize_k", "lazy_plain_decode_attn", "lazy_plain_prefill_attn",
     "lazy_debug_decode_table", "lazy_decode_attn_noalloc", "lazy_decode_noalloc_capacity",
     "lazy_cache_create", "lazy_cache_destroy", "lazy_cache_access", "lazy_cache_contains", "lazy_cache_stats",
-    "lazy_mixed_attn",
+    "lazy_mixed_attn", "lazy_rope_theta", "lazy_rope_theta_llama31", "lazy_alibi_slopes",
 ]
 
 
@@ -117,6 +117,10 @@ def _load():
         "lazy_decode_noalloc_capacity": (_sz, []),
         "lazy_mixed_attn": (_i, [_cfgp, ctypes.POINTER(PrefillBatch), ctypes.POINTER(DecodeBatch), _vp, _vp, _vp, _i,
                                  _vp, _vp]),
+        "lazy_rope_theta": (_i, [ctypes.c_double, _i, _vp]),
+        "lazy_rope_theta_llama31": (_i, [ctypes.c_double, _i, ctypes.c_double, ctypes.c_double, ctypes.c_double,
+                                         ctypes.c_double, _vp]),
+        "lazy_alibi_slopes": (_i, [_i, _vp]),
         "lazy_cache_create": (_vp, [_i64]),
         "lazy_cache_destroy": (None, [_vp]),
         "lazy_cache_access": (_i, [_vp, ctypes.c_uint64, ctypes.c_int32, _vp]),
@@ -167,6 +171,30 @@ def pack_words(block: np.ndarray, offset: np.ndarray) -> np.ndarray:
     _check("lazy_pack_words", _lib.lazy_pack_words(block.ctypes.data, offset.ctypes.data, block.size,
                                                    out.ctypes.data))
     return out
+
+
+def rope_theta(base: float, head_dim: int) -> tuple[float, ...]:
+    """lazy_rope_theta: theta_i = base^(-2i/head_dim)."""
+    out = np.empty(max(int(head_dim) // 2, 1), np.float64)
+    _check("lazy_rope_theta", _lib.lazy_rope_theta(float(base), int(head_dim), out.ctypes.data))
+    return tuple(float(x) for x in out[: int(head_dim) // 2])
+
+
+def rope_theta_llama31(base: float, head_dim: int, factor: float, low_freq_factor: float,
+                       high_freq_factor: float, original_max_position: float) -> tuple[float, ...]:
+    """lazy_rope_theta_llama31: frequencies with Llama-3.1 scaling."""
+    out = np.empty(max(int(head_dim) // 2, 1), np.float64)
+    _check("lazy_rope_theta_llama31", _lib.lazy_rope_theta_llama31(
+        float(base), int(head_dim), float(factor), float(low_freq_factor), float(high_freq_factor),
+        float(original_max_position), out.ctypes.data))
+    return tuple(float(x) for x in out[: int(head_dim) // 2])
+
+
+def alibi_slopes(num_heads: int) -> tuple[float, ...]:
+    """lazy_alibi_slopes: the ALiBi paper's head slopes."""
+    out = np.empty(max(int(num_heads), 1), np.float64)
+    _check("lazy_alibi_slopes", _lib.lazy_alibi_slopes(int(num_heads), out.ctypes.data))
+    return tuple(float(x) for x in out[: int(num_heads)])
 
 
 def kv_write(cfg: Cfg, k_raw, v_raw, slot, local_j, k_pool, v_pool, blk_meta, d_status=None, stream=None):

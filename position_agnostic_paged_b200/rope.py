@@ -1,60 +1,34 @@
 """Position-encoding tables for the configuration: RoPE frequencies (`rope_theta`) and ALiBi head
 slopes (`alibi_slopes`).
 
-The kernels take their rotation frequencies from one host table per call:
-theta_i = base^(-2i/d) by default, or any table passed as `Cfg.rope_theta`.
-The deferred rotation itself does not change: every angle is a position
-difference times theta_i.
+The tables are computed by the library (lazy_rope_theta, lazy_rope_theta_llama31,
+lazy_alibi_slopes in include/lazy_attn.h); these functions only forward their arguments and
+keep the Llama-3.1 defaults.  The kernels take their rotation frequencies from one host table
+per call, so a RoPE variant is a different table, not a different kernel: every angle is a
+position difference times theta_i.
 """
 from __future__ import annotations
 
-import math
+from . import lazy_attn as la
 
 
 def default_theta(base: float = 500000.0, head_dim: int = 128) -> tuple[float, ...]:
     """theta_i = base^(-2i/head_dim) for the rotate-half pairs (i, i + head_dim/2)."""
-    return tuple(base ** (-2.0 * i / head_dim) for i in range(head_dim // 2))
+    return la.rope_theta(base, head_dim)
 
 
 def llama31_theta(base: float = 500000.0, head_dim: int = 128, factor: float = 8.0,
                   low_freq_factor: float = 1.0, high_freq_factor: float = 4.0,
                   original_max_position: int = 8192) -> tuple[float, ...]:
-    """Frequencies with Llama-3.1 scaling (the "llama3" rope type of the Llama 3.1 configuration).
-
-    Each default frequency f has wavelength 2*pi/f.  Short wavelengths (below
-    original_max_position / high_freq_factor) keep f; long ones (above
-    original_max_position / low_freq_factor) use f / factor; in between the
-    frequency moves linearly, in original_max_position / wavelength, from f / factor
-    at low_freq_factor to f at high_freq_factor.
-    """
-    short_limit = original_max_position / high_freq_factor
-    long_limit = original_max_position / low_freq_factor
-    out = []
-    for f in default_theta(base, head_dim):
-        wavelength = 2.0 * math.pi / f
-        if wavelength < short_limit:
-            out.append(f)
-        elif wavelength > long_limit:
-            out.append(f / factor)
-        else:
-            w = (original_max_position / wavelength - low_freq_factor) / (high_freq_factor - low_freq_factor)
-            out.append(w * f + (1.0 - w) * f / factor)
-    return tuple(out)
+    """Frequencies with Llama-3.1 scaling (the "llama3" rope type of the Llama 3.1 configuration),
+    with that configuration's constants as defaults."""
+    return la.rope_theta_llama31(base, head_dim, factor, low_freq_factor, high_freq_factor,
+                                 original_max_position)
 
 
 def alibi_slopes(num_heads: int) -> tuple[float, ...]:
-    """ALiBi head slopes (Press, Smith and Lewis, "Train Short, Test Long", 2022) for Cfg.alibi_slopes.
-
-    With n a power of two the slopes are r, r^2, ..., r^n for r = 2^(-8/n).  Any other head count
-    takes the slopes of the largest power of two p below it and tops them up with every second
-    slope (the 1st, 3rd, 5th, ...) of the 2p-head sequence.
-    """
-    def geometric(n):
-        r = 2.0 ** (-8.0 / n)
-        return [r ** (k + 1) for k in range(n)]
-
+    """ALiBi head slopes (Press, Smith and Lewis, "Train Short, Test Long", 2022); raises ValueError
+    for num_heads <= 0."""
     if num_heads <= 0:
         raise ValueError("num_heads must be positive")
-    p = 1 << (num_heads.bit_length() - 1)
-    return tuple(geometric(p) + geometric(2 * p)[::2][: num_heads - p])
-
+    return la.alibi_slopes(num_heads)

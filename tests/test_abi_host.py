@@ -140,6 +140,29 @@ def test_position_tables_agree_with_the_oracle_s_own():
         np.testing.assert_allclose(rope.alibi_slopes(n), oracle.alibi_slopes(n), rtol=1e-14, atol=0)
 
 
+def test_table_exports_against_the_oracle_over_parameters():
+    """lazy_rope_theta, lazy_rope_theta_llama31 and lazy_alibi_slopes called through the C ABI
+    against the oracle's own computations, over bases, head sizes and scaling parameters."""
+    for base, d in ((500000.0, 128), (10000.0, 64), (1.0e6, 256), (2.5, 8)):
+        np.testing.assert_allclose(la.rope_theta(base, d), base ** (-(2.0 * np.arange(d // 2)) / d),
+                                   rtol=1e-15, atol=0)
+    for args in ((500000.0, 128, 8.0, 1.0, 4.0, 8192.0), (10000.0, 64, 4.0, 1.0, 4.0, 2048.0),
+                 (500000.0, 128, 1.0, 1.0, 4.0, 8192.0), (1.0e6, 128, 32.0, 2.0, 8.0, 65536.0)):
+        np.testing.assert_allclose(la.rope_theta_llama31(*args), oracle.llama31_theta(*args), rtol=1e-14, atol=0)
+    for n in range(1, 129):
+        np.testing.assert_allclose(la.alibi_slopes(n), oracle.alibi_slopes(n), rtol=1e-14, atol=0)
+    # arguments outside each rule's domain are refused before anything is written
+    buf = np.full(64, 7.0)
+    for bad in ((1.0, 128), (500000.0, 127), (500000.0, 0), (float("nan"), 128)):
+        assert la._lib.lazy_rope_theta(bad[0], bad[1], buf.ctypes.data) == la.LAZY_EINVAL
+    for bad in ((500000.0, 128, 0.0, 1.0, 4.0, 8192.0), (500000.0, 128, 8.0, 4.0, 4.0, 8192.0),
+                (500000.0, 128, 8.0, 1.0, 4.0, 0.0)):
+        assert la._lib.lazy_rope_theta_llama31(*bad, buf.ctypes.data) == la.LAZY_EINVAL
+    assert la._lib.lazy_alibi_slopes(0, buf.ctypes.data) == la.LAZY_EINVAL
+    assert la._lib.lazy_alibi_slopes(4, None) == la.LAZY_EINVAL
+    assert (buf == 7.0).all()
+
+
 def test_header_is_plain_c_and_cxx(tmp_path):
     """The public header compiles as C99 and C++11 on its own, and its inline codec packs words as
     documented (a C program built against the header alone, no CUDA)."""
