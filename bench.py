@@ -350,6 +350,11 @@ def run_ours(args):
     del ds, pool
     torch.cuda.empty_cache()
 
+    # ---------------------------------------------------------------- decode with no shared documents
+    if not args.no_distinct:
+        result["decode_distinct"] = run_decode_distinct(args, world, peaks, peak_src, flush)
+        result["gpu_launches"] += 3 * args.steps
+
     # ---------------------------------------------------------------- prefill leg
     if not args.no_prefill:
         result["prefill"] = run_prefill(args, world, peaks, peak_src, flush)
@@ -432,6 +437,42 @@ def run_e2e(ds, pool, step, dec_bytes, args, world):
     rate, ms = whole_job(world, dec_bytes, total / args.steps)
     return {"value": round(rate / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 5),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def run_decode_distinct(args, world, peaks, peak_src, flush):
+    """The decode 8B step with no document shared across requests (512 distinct documents, 8 per
+    request): every logical K/V byte is a distinct byte in HBM, so L2 cannot serve repeats and the
+    logical-byte fraction of the HBM peak is the kernel's real HBM efficiency."""
+    from position_agnostic_paged_b200 import accounting
+    from position_agnostic_paged_b200 import workloads as W
+    from position_agnostic_paged_b200.runner import DevicePool, DeviceStep
+
+    wl = W.make("decode_8b_distinct")
+    step = wl.steps[0]
+    pool = DevicePool(wl).setup()
+    ds = DeviceStep(pool, step)
+    _prepare_step_writes(ds)
+    b = accounting.decode_kv_bytes(step.kv_len, wl.hkv, wl.d)
+
+    def st(ev):
+        ds.write_new_tokens_dev()
+        if ev is not None:
+            ev[0].record()
+        ds.attend()
+        if ev is not None:
+            ev[1].record()
+
+    total, inner = timed_steps(st, args.steps, args.warmup, flush, world, inner=True)
+    attn = max_over_ranks(world, float(np.mean(inner)))
+    if pool.status() != 0:
+        raise SystemExit(f"device status {pool.status()} after distinct-document decode steps")
+    gbs = b / (attn * 1e-3) / 1e9
+    return {"workload": "decode_8b_distinct: decode 8B shapes, 64 requests x 4161 keys, 8 documents per request "
+                        "drawn without replacement across the batch (no document shared)",
+            "kv_bytes": b, "attn_ms": round(attn, 5), "GB/s": round(gbs, 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peak_src,
+                         "traffic": traffic_for("decode_8b_distinct", "decode.cu")}}
 
 
 def _time_alibi(ds, args, flush, world) -> float:
@@ -722,6 +763,8 @@ def main():
     ap.add_argument("--no-compare", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-distinct", action="store_true",
+                    help="skip the decode step over documents shared by no two requests")
     ap.add_argument("--extended", action="store_true",
                     help="also time decode 70B (Zipf 1.2 and uniform) and the mixed 8B step (GQA, MQA)")
     ap.add_argument("--profile-case", choices=["prefill_small", "decode_small", "decode_mqa_small"],

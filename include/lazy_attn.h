@@ -177,9 +177,10 @@ int lazy_decode_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int3
  * than the capacity (lazy_decode_workspace_bytes(cfg, num_req, max_words) >
  * capacity).  The first call on each device looks up the array's device
  * address (cudaGetSymbolAddress), so make that first call before any stream
- * capture.  All calls share the array: calls that can overlap on the GPU
- * (different streams or host threads) race and must be serialised by the
- * caller. */
+ * capture; the address is looked up again when the device's current context
+ * changes (e.g. after cudaDeviceReset).  All calls share the array: calls
+ * that can overlap on the GPU (different streams or host threads) race and
+ * must be serialised by the caller. */
 int lazy_decode_attn_noalloc(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *q_pos, int num_req,
                              const uint32_t *table, const int32_t *table_indptr, int max_words,
                              const uint32_t *blk_meta, const uint16_t *k_pool, const uint16_t *v_pool,
@@ -373,6 +374,19 @@ int lazy_alibi_slopes(int num_heads, double *slopes);
 int lazy_debug_decode_table(const uint32_t *table, int64_t n_words, const uint32_t *blk_meta,
                             int num_blocks, int32_t *out_block, int32_t *out_slot, int32_t *out_pos,
                             int *d_status, void *stream);
+
+/* Exercises the bounded pipeline wait that every warp-specialised kernel of
+ * the library uses, without stalling a real pipeline: one CTA arms an
+ * mbarrier that nothing completes (complete = 0) and waits on it for at most
+ * `polls` polls (1 .. 2^24), as a consumer whose copy never lands would; the
+ * wait gives up, ORs LAZY_DSTATUS_TIMEOUT into *d_status and raises the CTA's
+ * abort flag, and a second role waiting on another barrier leaves through
+ * that flag.  result: device int32[2] -- result[0] = 1 if the first wait ran
+ * out, result[1] = 1 if the second role left through the abort flag.  With
+ * complete != 0 both barriers complete first: both waits succeed, result is
+ * {0, 0} and nothing is reported.  LAZY_EINVAL for a null result or a poll
+ * count outside 1 .. 2^24. */
+int lazy_debug_bounded_wait(uint32_t polls, int complete, int32_t *result, int *d_status, void *stream);
 
 /* Text for a host return code (static storage). */
 const char *lazy_strerror(int code);

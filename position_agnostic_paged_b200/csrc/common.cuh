@@ -69,10 +69,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 // Waits until the phase with the given parity has completed.  Returns false
-// (after kWaitPolls polls) if it never does.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitPolls; ++i)
+// (after `polls` polls, kWaitPolls by default) if it never does.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t polls = kWaitPolls) {
+    for (uint32_t i = 0; i < polls; ++i)
         if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+// Bounded wait of one role of a warp-specialised kernel that also gives up as
+// soon as another role has aborted (a shared flag, checked every 256 polls).
+// The role whose own wait runs out sets the flag and LAZY_DSTATUS_TIMEOUT.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                              int *d_status, uint32_t polls = kWaitPolls) {
+    for (uint32_t i = 0; i < polls; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255) == 255 && *abort_flag) return false;
+    }
+    *abort_flag = 1;
+    if (d_status) atomicOr(d_status, LAZY_DSTATUS_TIMEOUT);
     return false;
 }
 

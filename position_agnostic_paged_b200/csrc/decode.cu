@@ -23,7 +23,6 @@
 // identity and runs once; each score gets slope_h * (o + j - p) in log2 units,
 // with o + j from the table word and the block's local index, as the mask uses.
 #include <climits>
-#include <cstdlib>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -378,21 +377,10 @@ cudaError_t launch_decode_t(const CUtensorMap &tk, const CUtensorMap &tv, const 
     return cudaGetLastError();
 }
 
-// Pipeline depth (8 KiB stages per CTA, a multiple of 4); LAZY_ATTN_DECODE_STAGES
-// selects 4, 8 or 12 for tuning experiments.
-int decode_stages() {
-    const char *env = getenv("LAZY_ATTN_DECODE_STAGES");
-    const int v = env ? atoi(env) : kDefaultStages;
-    return (v == 4 || v == 12) ? v : kDefaultStages;
-}
-
+// Pipeline depth: kDefaultStages stages of 8 KiB per CTA (a multiple of 4).
 template <int NT, bool PLAIN>
 cudaError_t launch_decode_nt(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, cudaStream_t s) {
-    switch (decode_stages()) {
-    case 4: return launch_decode_t<NT, PLAIN, 4>(tk, tv, p, s);
-    case 12: return launch_decode_t<NT, PLAIN, 12>(tk, tv, p, s);
-    default: return launch_decode_t<NT, PLAIN, kDefaultStages>(tk, tv, p, s);
-    }
+    return launch_decode_t<NT, PLAIN, kDefaultStages>(tk, tv, p, s);
 }
 
 }  // namespace
@@ -406,9 +394,7 @@ DecodePlan decode_plan(int num_req, int hkv, int max_words) {
     int splits = (target + units - 1) / units;
     const int max_splits = max(1, (max_words + 7) / 8);
     splits = max(1, min(splits, max_splits));
-    const char *env = getenv("LAZY_ATTN_DECODE_SPLIT_WORDS");
-    int wps = max(1, (max_words + splits - 1) / splits);
-    if (env && atoi(env) > 0) wps = atoi(env);
+    const int wps = max(1, (max_words + splits - 1) / splits);
     pl.words_per_split = wps;
     pl.n_splits = max(1, (max_words + wps - 1) / wps);
     return pl;

@@ -32,20 +32,49 @@ constexpr int kMaxDevices = 64;
 __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
 std::mutex g_mu;
-void *g_scratch_addr[kMaxDevices] = {};
+struct ScratchAddr {
+    void *ctx = nullptr;    // the context the address was looked up in
+    void *addr = nullptr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices];
 
-// Device address of the scratch array on the current device, looked up once
-// per device (the first call on a device does this set-up).
+typedef int (*CtxGetCurrentFn)(void **);
+
+// The driver's cuCtxGetCurrent, found once through the runtime (no link-time
+// dependency on libcuda); null if the driver does not provide it.
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    });
+    return fn;
+}
+
+// Device address of the scratch array in the current device's current
+// context.  It is looked up once per context (the first call on a device does
+// this set-up) and looked up again when the context changes -- after a
+// cudaDeviceReset the module may load at another address.  Without the
+// driver's context query the address is looked up on every call.
 int scratch_for_current_device(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LAZY_ECUDA;
+    void *ctx = nullptr;
+    CtxGetCurrentFn get = ctx_get_current();
+    const bool have_ctx = get && get(&ctx) == 0 && ctx;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_addr[dev]) {
+    ScratchAddr &e = g_scratch_addr[dev];
+    if (!have_ctx || !e.addr || e.ctx != ctx) {
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return LAZY_ECUDA;
-        g_scratch_addr[dev] = ptr;
+        e.addr = ptr;
+        e.ctx = have_ctx ? ctx : nullptr;
     }
-    *out = g_scratch_addr[dev];
+    *out = e.addr;
     return LAZY_OK;
 }
 
@@ -66,8 +95,9 @@ extern "C" int lazy_decode_attn_noalloc(const lazy_attn_cfg *cfg, const uint16_t
     void *scratch = nullptr;
     const int rc = scratch_for_current_device(&scratch);
     if (rc != LAZY_OK) return rc;
-    // The split partials are fully written before they are read, so the
-    // leftover contents of an earlier call need no clearing.
+    // Every split of every (request, KV head) writes its partial (an empty
+    // split writes m = -inf, l = 0 and a zero accumulator) before the combine
+    // reads it, so the leftover contents of an earlier call need no clearing.
     return lazy_decode_attn(cfg, q_raw, q_pos, num_req, table, table_indptr, max_words, blk_meta, k_pool, v_pool,
                             num_blocks, out, scratch, kStaticScratchBytes, d_status, stream);
 }

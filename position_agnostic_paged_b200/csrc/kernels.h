@@ -82,6 +82,7 @@ DecodePlan decode_plan(int num_req, int hkv, int max_words);
 cudaError_t launch_kv_write(const KvWriteParams &p, cudaStream_t s);
 cudaError_t launch_decode_table(const DecodeTableParams &p, cudaStream_t s);
 cudaError_t launch_materialize(const MaterializeParams &p, cudaStream_t s);
+cudaError_t launch_debug_bounded_wait(uint32_t polls, int complete, int *result, int *d_status, cudaStream_t s);
 cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, bool plain,
                           cudaStream_t s);
 // tk, tv: the K source and V pool as rows of 128 bf16 (one box = half of one block);

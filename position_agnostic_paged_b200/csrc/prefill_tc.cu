@@ -98,17 +98,6 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Bounded wait that also gives up as soon as another role has aborted.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                              int *d_status) {
-    for (uint32_t i = 0; i < kWaitPolls; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255) == 255 && *abort_flag) return false;
-    }
-    *abort_flag = 1;
-    set_status(d_status, LAZY_DSTATUS_TIMEOUT);
-    return false;
-}
 // 4D tiled load: 8 consecutive blocks of one head, one 64-element half (16 KiB).
 __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int x, int y, int h, int b,
                                             uint64_t *bar) {

@@ -28,6 +28,7 @@ EXPORTED = [
     "lazy_debug_decode_table", "lazy_decode_attn_noalloc", "lazy_decode_noalloc_capacity",
     "lazy_cache_create", "lazy_cache_destroy", "lazy_cache_access", "lazy_cache_contains", "lazy_cache_stats",
     "lazy_mixed_attn", "lazy_rope_theta", "lazy_rope_theta_llama31", "lazy_alibi_slopes",
+    "lazy_debug_bounded_wait",
 ]
 
 
@@ -121,6 +122,7 @@ def _load():
         "lazy_rope_theta_llama31": (_i, [ctypes.c_double, _i, ctypes.c_double, ctypes.c_double, ctypes.c_double,
                                          ctypes.c_double, _vp]),
         "lazy_alibi_slopes": (_i, [_i, _vp]),
+        "lazy_debug_bounded_wait": (_i, [ctypes.c_uint32, _i, _vp, _vp, _vp]),
         "lazy_cache_create": (_vp, [_i64]),
         "lazy_cache_destroy": (None, [_vp]),
         "lazy_cache_access": (_i, [_vp, ctypes.c_uint64, ctypes.c_int32, _vp]),
@@ -298,6 +300,12 @@ def debug_decode_table(table, blk_meta, num_blocks: int, out_block, out_slot, ou
     _check("lazy_debug_decode_table", _lib.lazy_debug_decode_table(
         _ptr(table), int(table.numel()), _ptr(blk_meta), int(num_blocks), _ptr(out_block), _ptr(out_slot),
         _ptr(out_pos), _ptr(d_status), _stream(stream)))
+
+
+def debug_bounded_wait(polls: int, complete: bool, result, d_status=None, stream=None):
+    """lazy_debug_bounded_wait: a bounded mbarrier wait that runs out (complete=False) or succeeds."""
+    _check("lazy_debug_bounded_wait", _lib.lazy_debug_bounded_wait(
+        int(polls), 1 if complete else 0, _ptr(result), _ptr(d_status), _stream(stream)))
 
 
 def decode_noalloc_capacity() -> int:

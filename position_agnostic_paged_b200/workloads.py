@@ -197,7 +197,8 @@ def build_rag(*, name: str, seed: int, hq: int, hkv: int, d: int = 128, rope_bas
               n_docs: int, doc_len, docs_per_req: int, alpha: float, n_prefill: int = 0,
               prefill_len: int = 256, n_decode: int = 0, question_len: int = 64,
               decode_steps: int = 1, pool_cap_blocks: int | None = None,
-              prefill_docs_per_req: int | None = None, uniform_docs: bool = False) -> Workload:
+              prefill_docs_per_req: int | None = None, uniform_docs: bool = False,
+              distinct_docs: bool = False) -> Workload:
     """General RAG workload: prefill chunks and/or decode requests over a shared pool.
 
     doc_len: an int (every document that long) or a (lo, hi) pair (uniform).
@@ -208,6 +209,9 @@ def build_rag(*, name: str, seed: int, hq: int, hkv: int, d: int = 128, rope_bas
     pool_cap_blocks: if set, the pool holds at most that many blocks in total
     (questions included); the document population is the popularity-ranked
     prefix of documents that fits.
+    distinct_docs: draw the documents of all requests together, without
+    replacement, so that no document is shared by two requests (every logical
+    K/V byte of the step is then a distinct physical byte).
     """
     rng0 = np.random.default_rng([seed, 0])
     pf_docs = prefill_docs_per_req if prefill_docs_per_req is not None else docs_per_req
@@ -236,8 +240,16 @@ def build_rag(*, name: str, seed: int, hq: int, hkv: int, d: int = 128, rope_bas
         sel = rng0.choice(n_docs, size=k, replace=False, p=p)
         return [int(x) for x in rng0.permutation(sel)]
 
-    pf_draws = [draw(pf_docs) for _ in range(n_prefill)]
-    dec_draws = [draw(docs_per_req) for _ in range(n_decode)]
+    if distinct_docs:
+        need = n_prefill * pf_docs + n_decode * docs_per_req
+        assert need <= n_docs, "distinct documents: the pool is too small"
+        allsel = [int(x) for x in rng0.choice(n_docs, size=need, replace=False, p=p)]
+        pf_draws = [allsel[i * pf_docs:(i + 1) * pf_docs] for i in range(n_prefill)]
+        base = n_prefill * pf_docs
+        dec_draws = [allsel[base + i * docs_per_req: base + (i + 1) * docs_per_req] for i in range(n_decode)]
+    else:
+        pf_draws = [draw(pf_docs) for _ in range(n_prefill)]
+        dec_draws = [draw(docs_per_req) for _ in range(n_decode)]
 
     used = sorted(set(x for dd in pf_draws + dec_draws for x in dd))
     bld = _Builder(hkv, d)
@@ -353,6 +365,9 @@ CONFIGS = {
                       n_decode=64, question_len=64),
     "prefill_8b": dict(hq=32, hkv=8, n_docs=1000, doc_len=512, docs_per_req=10, alpha=1.0,
                        n_prefill=16, prefill_len=256),
+    # decode 8B with no document shared across requests: 512 of the 1000 documents, each in one request
+    "decode_8b_distinct": dict(hq=32, hkv=8, n_docs=1000, doc_len=512, docs_per_req=8, alpha=1.0,
+                               n_decode=64, question_len=64, distinct_docs=True),
     "decode_70b": dict(hq=64, hkv=8, n_docs=4000, doc_len=512, docs_per_req=32, alpha=1.2,
                        n_decode=128, question_len=128),
     "decode_70b_uniform": dict(hq=64, hkv=8, n_docs=4000, doc_len=512, docs_per_req=32, alpha=0.0,
@@ -367,7 +382,7 @@ CONFIGS = {
 
 # seeds: 1000 + the configuration's index in the order tiny, decode 8B,
 # prefill 8B, decode 70B, mixed 8B
-SEEDS = {"tiny": 1001, "decode_8b": 1002, "prefill_8b": 1003, "decode_70b": 1004,
+SEEDS = {"tiny": 1001, "decode_8b": 1002, "decode_8b_distinct": 1002, "prefill_8b": 1003, "decode_70b": 1004,
          "decode_70b_uniform": 1004, "mixed_8b": 1005, "mixed_8b_mqa": 1005}
 
 

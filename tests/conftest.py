@@ -27,3 +27,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Measured parity errors of this session (one line per comparison)."""
+    from tests._report import RESULTS
+    if not RESULTS:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", f"parity errors ({len(RESULTS)} comparisons)")
+    worst = max(r[1] / r[3] for r in RESULTS)
+    tr.write_line(f"largest max_abs / bound: {worst:.3f}")
+    for what, ma, rl, ba, br in RESULTS:
+        tr.write_line(f"{what:<60s} max_abs {ma:.3e} (<= {ba:.1e})  rel_l2 {rl:.3e} (<= {br:.1e})")

@@ -14,6 +14,7 @@ from position_agnostic_paged_b200 import workloads as W
 from position_agnostic_paged_b200.runner import DevicePool, DeviceStep
 from tests._cases import bits_to_f64, make_case
 from tests._gpu_cases import DeviceCase
+from tests._report import record
 
 pytestmark = pytest.mark.gpu
 
@@ -39,6 +40,7 @@ def check(got, ref, max_abs=MAX_ABS, rel_l2=REL_L2, what=""):
     err = np.abs(got - ref)
     ma = float(err.max()) if err.size else 0.0
     rl = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+    record(what, ma, rl, max_abs, rel_l2)
     assert ma <= max_abs and rl <= rel_l2, f"{what}: max_abs={ma:.3e} rel_l2={rl:.3e}"
     return ma, rl
 
@@ -519,9 +521,19 @@ def _sample_rows(step, hq, n, seed):
     return q.astype(np.int32), h.astype(np.int32)
 
 
-def _run_full(name, n_rows, **over):
+def _chunk_rows(step, hq, requests):
+    """Every (query, head) row of the given requests of a prefill step."""
+    q = np.concatenate([np.arange(step.cu_q[r], step.cu_q[r + 1]) for r in requests]).astype(np.int32)
+    return np.repeat(q, hq), np.tile(np.arange(hq, dtype=np.int32), q.size)
+
+
+def _run_full(name, prefill_requests=None, **over):
+    """The named workload at full size in the launch configuration the benchmark times: lazy and
+    plain outputs against the oracle on EVERY output row (for a prefill step with
+    prefill_requests given, every row of those requests), and lazy against plain on every row."""
     wl = W.make(name, **over)
     pool = DevicePool(wl).setup()
+    tag = name + "".join(f" {k}={v}" for k, v in over.items())
     results = []
     for step in wl.steps:
         ds = DeviceStep(pool, step, with_plain=True)
@@ -530,25 +542,78 @@ def _run_full(name, n_rows, **over):
         ds.materialize()
         ds.attend_plain()
         torch.cuda.synchronize()
-        sq, sh = _sample_rows(step, wl.hq, n_rows, 7)
-        ref = oracle_step(wl, step, sq, sh)
         lazy = ds.out_f64().reshape(step.total_q, wl.hq, wl.d)
         plain = ds.out_f64(ds.out_plain).reshape(step.total_q, wl.hq, wl.d)
-        check(lazy[sq, sh], ref, what=f"{name} {step.kind} sampled lazy")
-        check(plain[sq, sh], ref, what=f"{name} {step.kind} sampled plain")
+        if step.kind == "prefill" and prefill_requests is not None:
+            sq, sh = _chunk_rows(step, wl.hq, prefill_requests)
+            ref = oracle_step(wl, step, sq, sh)
+            what = f"{tag} {step.kind} (every row of requests {list(prefill_requests)})"
+            check(lazy[sq, sh], ref, what=f"{what} lazy")
+            check(plain[sq, sh], ref, what=f"{what} plain")
+        else:
+            ref = oracle_step(wl, step)
+            check(lazy.reshape(-1, wl.d), ref, what=f"{tag} {step.kind} every row, lazy")
+            check(plain.reshape(-1, wl.d), ref, what=f"{tag} {step.kind} every row, plain")
         # every row: lazy and materialised paths agree (a property that holds at any size)
-        check(lazy.reshape(-1, wl.d), plain.reshape(-1, wl.d), what=f"{name} {step.kind} lazy vs plain")
+        check(lazy.reshape(-1, wl.d), plain.reshape(-1, wl.d), what=f"{tag} {step.kind} lazy vs plain")
         results.append(step.kind)
     assert pool.status() == 0
     return results
 
 
 def test_decode_8b_full_size():
-    assert _run_full("decode_8b", 64) == ["decode"]
+    assert _run_full("decode_8b") == ["decode"]
 
 
 def test_prefill_8b_full_size():
-    assert _run_full("prefill_8b", 64) == ["prefill"]
+    assert _run_full("prefill_8b") == ["prefill"]
+
+
+def test_materialized_keys_against_the_oracle():
+    """lazy_materialize_k writes bf16(RoPE(stored key, o)) for every table word: keys re-encoded at
+    their absolute positions.  The oracle rotates the raw key once to o + j in fp64 and rounds once;
+    the kernel starts from the pool's key (already rounded at j) and rounds again, so each element
+    may differ by the first rounding carried through the rotation plus the second: at most
+    2^-8 r + 2^-9 |k'| (+ 2^-20 for fp32 arithmetic), r = the pair's radius sqrt(k_i^2 + k_(i+64)^2),
+    and most elements agree to one ulp."""
+    wl = W.make("decode_8b", n_decode=8, n_docs=100)
+    pool = DevicePool(wl).setup()
+    step = wl.steps[0]
+    ds = DeviceStep(pool, step, with_plain=True)
+    ds.write_new_tokens()
+    ds.materialize()
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    got = ds.k_mat.view(torch.int16).cpu().numpy().view(np.uint16)         # [word, head, slot, d]
+    # store row of every pool slot, and each word's slots' logical positions, from the oracle's own
+    # pool metadata and table expansion
+    row_of_slot = np.full(wl.num_blocks * 16, -1, np.int64)
+    row_of_slot[wl.store_slot] = np.arange(wl.store_slot.size)
+    written = np.concatenate([wl.setup_rows, step.write_rows])
+    meta = np.zeros(wl.num_blocks, np.uint32)
+    scratch = np.zeros((wl.num_blocks, wl.hkv, 16, wl.d), np.uint16)
+    assert oracle.kv_write(wl.k_store[written], wl.v_store[written], wl.store_slot[written], wl.store_j[written],
+                           scratch, scratch.copy(), meta, wl.rope_base) == 0
+    words = np.array([oracle.pack_word(b, o) for b, o in zip(step.table_block, step.table_off)], np.uint32)
+    eb, es, epos, rc = oracle.expand_table(words, meta, wl.num_blocks)
+    assert rc == 0
+    valid = epos.ravel() >= 0
+    rows = row_of_slot[es.ravel()[valid]]
+    assert (rows >= 0).all()
+    want = oracle.rope_rows_bf16(wl.k_store[rows], epos.ravel()[valid].astype(np.int32), wl.rope_base)
+    g = got.transpose(0, 2, 1, 3).reshape(-1, wl.hkv, wl.d)[valid]           # [valid slot, head, d]
+    gf, wf = bits_to_f64(g), bits_to_f64(want)
+    kr = bits_to_f64(wl.k_store[rows])
+    radius = np.sqrt(kr[..., :64] ** 2 + kr[..., 64:] ** 2)
+    radius = np.concatenate([radius, radius], axis=-1)
+    bound = 2.0 ** -8 * radius + 2.0 ** -9 * np.abs(wf) + 2.0 ** -20
+    err = np.abs(gf - wf)
+    assert (err <= bound).all(), f"max err/bound {float((err / bound).max()):.3f}"
+    ulps = np.abs(g.astype(np.int32) - want.astype(np.int32))
+    assert (ulps <= 1).mean() > 0.95, f"{(ulps <= 1).mean():.4f} within one ulp"
+    # slots past n_valid are written as zeros
+    assert (got.transpose(0, 2, 1, 3).reshape(-1, wl.hkv, wl.d)[~valid] == 0).all()
+    record("materialised keys vs oracle (err / bound)", float((err / bound).max()), 0.0, 1.0, 0.0)
 
 
 @pytest.mark.parametrize("name", ["decode_8b", "prefill_8b"])
@@ -606,9 +671,23 @@ def test_mixed_step_full_size():
 
 @pytest.mark.slow
 def test_decode_70b_full_size():
-    assert _run_full("decode_70b", 24) == ["decode"]
+    assert _run_full("decode_70b") == ["decode"]
+
+
+@pytest.mark.slow
+def test_decode_70b_uniform_full_size():
+    """The uniform-popularity variant of decode 70B (alpha = 0): little sharing across requests."""
+    assert _run_full("decode_70b_uniform") == ["decode"]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("alpha", [0.6, 1.0, 1.4])
+def test_mixed_8b_alpha_sweep(alpha):
+    """The mixed 8B step at each Zipf exponent of the sweep: every decode row, and every row of four
+    of the 32 prefill chunks (the first, the last and two between), against the oracle."""
+    assert _run_full("mixed_8b", prefill_requests=(0, 11, 22, 31), alpha=alpha) == ["prefill", "decode"]
 
 
 @pytest.mark.slow
 def test_mixed_8b_mqa_full_size():
-    assert _run_full("mixed_8b_mqa", 32) == ["prefill", "decode"]
+    assert _run_full("mixed_8b_mqa", prefill_requests=(0, 15, 31)) == ["prefill", "decode"]

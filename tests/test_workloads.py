@@ -87,3 +87,17 @@ def test_inputs_are_seeded_and_deterministic():
     assert np.array_equal(sa.seg_src, sb.seg_src) and np.array_equal(a.k_store[:4096], b.k_store[:4096])
     c = W.make("decode_8b", seed=7)
     assert not np.array_equal(c.steps[0].seg_src, sa.seg_src)
+
+
+def test_distinct_decode_workload_shares_no_document():
+    """decode_8b_distinct: the decode 8B shapes with every document in exactly one request, so the
+    step's logical K/V bytes are all distinct physical bytes."""
+    wl = W.make("decode_8b_distinct", n_decode=8)
+    st = wl.steps[0]
+    seen = set()
+    for r in range(st.num_req):
+        blocks = set(st.table_block[st.table_indptr[r]:st.table_indptr[r + 1]].tolist())
+        assert not (blocks & seen)
+        seen |= blocks
+    assert wl.info["unique_docs_used"] == 8 * 8
+    assert (st.kv_len == 8 * 512 + 65).all()
