@@ -22,17 +22,47 @@ MAX_ABS = 1e-2
 REL_L2 = 5e-3
 
 
-def edge_max_abs(case) -> float:
-    """Absolute bound for hand-made cases where a query may see only a few keys.
+FEW_KEYS = 16
 
-    The kernels feed P to the PV product in bf16 (relative rounding <= 2^-9
-    per weight) and round the output to bf16 (<= 2^-9 |O|).  With few visible
-    keys O is close to single value rows, so the error is bounded by about
-    2^-9 (|O| + 2 max|V|) <= 3 * 2^-9 * max|V| -- the config-sized workloads,
-    where every query sees thousands of keys, keep the absolute 1e-2.
-    """
+
+def visible_keys(case) -> np.ndarray:
+    """Keys each output row's query sees (rows q-major, head-minor), from the case's segments."""
+    n_q = case.q_pos.size
+    vis = np.zeros(n_q, np.int64)
+    for r in range(case.cu_q.size - 1):
+        for q in range(case.cu_q[r], case.cu_q[r + 1]):
+            p = int(case.q_pos[q])
+            for g in range(case.seg_indptr[r], case.seg_indptr[r + 1]):
+                vis[q] += max(0, min(int(case.seg_len[g]), p - int(case.seg_off[g]) + 1))
+    return np.repeat(vis, case.hq)
+
+
+def few_keys_bound(case) -> float:
+    """Absolute bound for output rows whose query sees fewer than FEW_KEYS keys.
+
+    Such a row is close to a few value rows, so |O| can reach max|V|, and the bf16 steps of
+    the kernels do not average out: the output is rounded to bf16 (up to 2^-8 |O|) and each
+    softmax weight fed to the PV product is rounded to bf16 (relative 2^-8, up to
+    2^-8 * 2 max|V| on O).  The worst case is 3 * 2^-8 * max|V|; the bound used is half of
+    it, 1.5 * 2^-8 * max|V| (about 0.026 for N(0,1) values), which every such row meets with
+    margin (the measured errors are recorded by the session summary).  Rows that see
+    FEW_KEYS keys or more keep the absolute 1e-2."""
     vmax = float(np.abs(bits_to_f64(case.v_tok)).max())
-    return max(MAX_ABS, 3 * 2.0 ** -9 * vmax)
+    return max(MAX_ABS, 1.5 * 2.0 ** -8 * vmax)
+
+
+def check_case(got, ref, case, what="", rel_l2=REL_L2):
+    """check() for a hand-made case: 1e-2 on rows that see FEW_KEYS keys or more,
+    few_keys_bound(case) on the others, and rel-L2 over the whole output."""
+    vis = visible_keys(case)
+    assert vis.size == got.shape[0] == ref.shape[0]
+    many = vis >= FEW_KEYS
+    if many.any():
+        check(got[many], ref[many], max_abs=MAX_ABS, rel_l2=np.inf, what=f"{what} [rows seeing >= {FEW_KEYS} keys]")
+    if (~many).any():
+        check(got[~many], ref[~many], max_abs=few_keys_bound(case), rel_l2=np.inf,
+              what=f"{what} [rows seeing < {FEW_KEYS} keys]")
+    return check(got, ref, max_abs=max(MAX_ABS, few_keys_bound(case)), rel_l2=rel_l2, what=f"{what} [all rows]")
 
 
 def check(got, ref, max_abs=MAX_ABS, rel_l2=REL_L2, what=""):
@@ -168,12 +198,11 @@ def test_adversarial_cases_all_group_sizes(kind, hq, hkv):
     case = make_case(100 + hq + hkv, hq=hq, hkv=hkv, d=128, requests=_adv_requests(kind == "decode"))
     dc = DeviceCase(case)
     ref = oracle.attend(**case.oracle_kwargs())
-    tol = edge_max_abs(case)
     split = kind == "prefill"
     got = dc.decode() if kind == "decode" else dc.prefill(split=split)
-    check(got, ref, max_abs=tol, what=f"{kind} G={hq // hkv} lazy")
+    check_case(got, ref, case, what=f"{kind} G={hq // hkv} lazy")
     got_p = dc.decode(plain=True) if kind == "decode" else dc.prefill(plain=True, split=split)
-    check(got_p, ref, max_abs=tol, what=f"{kind} G={hq // hkv} plain")
+    check_case(got_p, ref, case, what=f"{kind} G={hq // hkv} plain")
     assert dc.status() == 0
 
 
@@ -195,11 +224,10 @@ def test_scattered_document_blocks(kind, scatter):
     case = make_case(31, hq=32, hkv=8, d=128, requests=_long_requests(kind == "decode"))
     dc = DeviceCase(case, scatter_seed=scatter)
     ref = oracle.attend(**case.oracle_kwargs())
-    tol = edge_max_abs(case)
     got = dc.decode() if kind == "decode" else dc.prefill()
-    check(got, ref, max_abs=tol, what=f"{kind} scatter={scatter} lazy")
+    check_case(got, ref, case, what=f"{kind} scatter={scatter} lazy")
     got_p = dc.decode(plain=True) if kind == "decode" else dc.prefill(plain=True)
-    check(got_p, ref, max_abs=tol, what=f"{kind} scatter={scatter} plain")
+    check_case(got_p, ref, case, what=f"{kind} scatter={scatter} plain")
     assert dc.status() == 0
 
 
@@ -214,7 +242,7 @@ def test_offsets_near_the_15_bit_limit(kind):
     dc = DeviceCase(case)
     ref = oracle.attend(**case.oracle_kwargs())
     got = dc.decode() if kind == "decode" else dc.prefill()
-    check(got, ref, max_abs=edge_max_abs(case), what=f"{kind} offsets near 2^15")
+    check_case(got, ref, case, what=f"{kind} offsets near 2^15")
     assert dc.status() == 0
 
 
@@ -230,7 +258,7 @@ def test_block_ids_near_the_17_bit_limit(kind):
     assert int(dc.phys[:nb].max()) > (1 << 16)
     ref = oracle.attend(**case.oracle_kwargs())
     got = dc.decode() if kind == "decode" else dc.prefill()
-    check(got, ref, max_abs=edge_max_abs(case), what=f"{kind} block ids near 2^17")
+    check_case(got, ref, case, what=f"{kind} block ids near 2^17")
     assert dc.status() == 0
 
 
@@ -243,7 +271,7 @@ def test_request_with_an_empty_table_among_others():
     ref = oracle.attend(**case.oracle_kwargs())
     out = dc.decode()
     assert np.array_equal(out[32:64], np.zeros((32, 128)))
-    check(out, ref, max_abs=edge_max_abs(case), what="decode with an empty table")
+    check_case(out, ref, case, what="decode with an empty table")
     assert dc.status() == 0
 
 
@@ -254,8 +282,8 @@ def test_prefill_request_with_no_query_tokens():
     case = make_case(53, hq=32, hkv=8, d=128, requests=reqs)
     dc = DeviceCase(case)
     ref = oracle.attend(**case.oracle_kwargs())
-    check(dc.prefill(), ref, max_abs=edge_max_abs(case), what="prefill with an empty chunk")
-    check(dc.prefill(split=False), ref, max_abs=edge_max_abs(case), what="prefill with an empty chunk, unsplit")
+    check_case(dc.prefill(), ref, case, what="prefill with an empty chunk")
+    check_case(dc.prefill(split=False), ref, case, what="prefill with an empty chunk, unsplit")
     assert dc.status() == 0
 
 
@@ -280,12 +308,12 @@ def test_llama31_frequency_table(kind):
     case = make_case(61, hq=32, hkv=8, d=128, requests=[(segs, qp)])
     dc = DeviceCase(case, rope_theta=tp)
     ref = oracle.attend(**case.oracle_kwargs(), rope_theta=to)
-    tol = edge_max_abs(case)
+    tol = few_keys_bound(case)
     assert np.abs(ref - oracle.attend(**case.oracle_kwargs())).max() > 3 * tol   # the table matters here
     got = dc.decode() if kind == "decode" else dc.prefill()
-    check(got, ref, max_abs=tol, what=f"{kind} llama-3.1 frequencies, lazy")
+    check_case(got, ref, case, what=f"{kind} llama-3.1 frequencies, lazy")
     got_p = dc.decode(plain=True) if kind == "decode" else dc.prefill(plain=True)
-    check(got_p, ref, max_abs=tol, what=f"{kind} llama-3.1 frequencies, plain")
+    check_case(got_p, ref, case, what=f"{kind} llama-3.1 frequencies, plain")
     assert dc.status() == 0
 
 
@@ -357,10 +385,10 @@ def test_alibi_attention(kind, hq, hkv):
     case = make_case(200 + hq + hkv, hq=hq, hkv=hkv, d=128, requests=_adv_requests(kind == "decode"))
     dc = DeviceCase(case, alibi_slopes=sp)
     ref = oracle.attend(**case.oracle_kwargs(), alibi_slopes=so)
-    tol = edge_max_abs(case)
+    tol = few_keys_bound(case)
     assert np.abs(ref - oracle.attend(**case.oracle_kwargs())).max() > 3 * tol   # the encoding matters
     got = dc.decode() if kind == "decode" else dc.prefill(split=kind == "prefill")
-    check(got, ref, max_abs=tol, what=f"{kind} G={hq // hkv} alibi")
+    check_case(got, ref, case, what=f"{kind} G={hq // hkv} alibi")
     assert dc.status() == 0
 
 
@@ -375,7 +403,7 @@ def test_alibi_long_context_and_full_tiles(kind):
     dc = DeviceCase(case, alibi_slopes=sp)
     ref = oracle.attend(**case.oracle_kwargs(), alibi_slopes=so)
     got = dc.decode() if kind == "decode" else dc.prefill()
-    check(got, ref, max_abs=edge_max_abs(case), what=f"{kind} alibi long")
+    check_case(got, ref, case, what=f"{kind} alibi long")
     assert dc.status() == 0
 
 
@@ -432,9 +460,8 @@ def test_mixed_step_equals_separate_calls_and_the_oracle(hq, hkv):
     assert torch.equal(pf["out"], pf2["out"]) and torch.equal(dc["out"], dc2["out"])
     ref = oracle.attend(**case.oracle_kwargs())
     n_pf = int(case.cu_q[3]) * hq
-    tol = edge_max_abs(case)
-    check(_f64(pf["out"]), ref[:n_pf], max_abs=tol, what="mixed: prefill part")
-    check(_f64(dc["out"]), ref[n_pf:], max_abs=tol, what="mixed: decode part")
+    got = np.concatenate([_f64(pf["out"]), _f64(dc["out"])])
+    check_case(got, ref, case, what=f"mixed step G={hq // hkv} (prefill rows then decode rows)")
     assert dc_.status() == 0
 
 
@@ -484,7 +511,8 @@ def test_queries_that_see_nothing_give_zero_rows():
     dc = DeviceCase(case)
     out = dc.decode()
     assert np.array_equal(out[:8], np.zeros((8, 128)))
-    check(out[8:], oracle.attend(**case.oracle_kwargs())[8:], max_abs=edge_max_abs(case))
+    ref = oracle.attend(**case.oracle_kwargs())
+    check_case(out, ref, case, what="queries that see nothing")
 
 
 def test_peaked_scores():
@@ -496,7 +524,7 @@ def test_peaked_scores():
     ref = oracle.attend(**case.oracle_kwargs())
     # score errors scale with |q|: bf16 rounding of q' and k (2^-9 relative
     # each) on scores 4x larger; the bound below is 4x the base tolerance
-    check(dc.decode(), ref, max_abs=4 * edge_max_abs(case), rel_l2=2e-2, what="peaked decode")
+    check(dc.decode(), ref, max_abs=4 * few_keys_bound(case), rel_l2=2e-2, what="peaked decode")
 
 
 def test_decode_equals_last_prefill_row():
@@ -572,10 +600,12 @@ def test_prefill_8b_full_size():
 def test_materialized_keys_against_the_oracle():
     """lazy_materialize_k writes bf16(RoPE(stored key, o)) for every table word: keys re-encoded at
     their absolute positions.  The oracle rotates the raw key once to o + j in fp64 and rounds once;
-    the kernel starts from the pool's key (already rounded at j) and rounds again, so each element
-    may differ by the first rounding carried through the rotation plus the second: at most
-    2^-8 r + 2^-9 |k'| (+ 2^-20 for fp32 arithmetic), r = the pair's radius sqrt(k_i^2 + k_(i+64)^2),
-    and most elements agree to one ulp."""
+    the kernel starts from the pool's key (already rounded at j) and rounds again.  With the bf16
+    unit roundoff u = 2^-8, the first rounding moves each component of the pair by at most
+    u * r (r = the pair's radius sqrt(k_i^2 + k_(i+64)^2), which the rotations preserve), and the
+    rotation mixes the two components, so it reaches an element as at most sqrt(2) u r; the second
+    rounding adds u |k'|.  Bound: sqrt(2) u r + u |k'| + 2^-20 (fp32 arithmetic); most elements
+    agree to one ulp."""
     wl = W.make("decode_8b", n_decode=8, n_docs=100)
     pool = DevicePool(wl).setup()
     step = wl.steps[0]
@@ -606,7 +636,7 @@ def test_materialized_keys_against_the_oracle():
     kr = bits_to_f64(wl.k_store[rows])
     radius = np.sqrt(kr[..., :64] ** 2 + kr[..., 64:] ** 2)
     radius = np.concatenate([radius, radius], axis=-1)
-    bound = 2.0 ** -8 * radius + 2.0 ** -9 * np.abs(wf) + 2.0 ** -20
+    bound = np.sqrt(2.0) * 2.0 ** -8 * radius + 2.0 ** -8 * np.abs(wf) + 2.0 ** -20
     err = np.abs(gf - wf)
     assert (err <= bound).all(), f"max err/bound {float((err / bound).max()):.3f}"
     ulps = np.abs(g.astype(np.int32) - want.astype(np.int32))
