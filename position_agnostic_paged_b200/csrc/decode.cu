@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_split_kernel(const _
 // holds the rows (heads) lane/4 and lane/4 + 8 of its tile: the raw query as bf16 pairs, the
 // rotated query fragments, 16 x 4 output accumulators and the two rows' softmax state.
 template <int MT, bool PLAIN, int kDecodeStages>
-__global__ void __launch_bounds__(kDecodeThreads, 2) decode_heads_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(kDecodeThreads, 3) decode_heads_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                       const __grid_constant__ CUtensorMap tmV,
                                                                       const AttnParams p) {
     constexpr int KW = 4 / MT;   // warps sharing the words of one head tile
@@ -404,18 +404,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_heads_kernel(const _
     } else {
         // raw query, A-fragment order: k-step s, register x: head (x & 1 ? h1 : h0), head-dim
         // elements 16s + 8(x >> 1) + 2c and + 1
-        uint32_t qr[8][4];
-        {
-            const uint16_t *qb = p.q_raw + (static_cast<size_t>(r) * p.hq + kvh * G) * kHeadDim;
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const int h = (x & 1) ? h1 : h0;
-                    qr[s][x] = h < G ? *reinterpret_cast<const uint32_t *>(qb + h * kHeadDim + 16 * s + 8 * (x >> 1) + 2 * c)
-                                     : 0u;
-                }
-        }
+        // raw query pairs of this thread, read from global memory (L1-resident after the first
+        // rotation) whenever the query is rotated, to keep registers for the accumulators
+        const uint16_t *qb = p.q_raw + (static_cast<size_t>(r) * p.hq + kvh * G) * kHeadDim;
+        auto qraw = [&](int s, int x) -> uint32_t {
+            const int h = (x & 1) ? h1 : h0;
+            return h < G ? __ldg(reinterpret_cast<const unsigned int *>(qb + h * kHeadDim + 16 * s + 8 * (x >> 1) + 2 * c))
+                         : 0u;
+        };
         uint32_t qf[8][4];
         int cur_off = INT_MIN;
         const float sl0 = slope_s[h0 < 32 ? h0 : 0], sl1 = slope_s[h1 < 32 ? h1 : 0];
@@ -452,9 +448,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_heads_kernel(const _
 #pragma unroll
                             for (int hr = 0; hr < 2; ++hr) {
                                 const int x = 2 * half + hr;
-                                const float a0 = bf16_lo(qr[s][x]) * p.scale_log2, a1 = bf16_hi(qr[s][x]) * p.scale_log2;
-                                const float b0 = bf16_lo(qr[s + 4][x]) * p.scale_log2,
-                                            b1 = bf16_hi(qr[s + 4][x]) * p.scale_log2;
+                                const uint32_t ra = qraw(s, x), rb = qraw(s + 4, x);
+                                const float a0 = bf16_lo(ra) * p.scale_log2, a1 = bf16_hi(ra) * p.scale_log2;
+                                const float b0 = bf16_lo(rb) * p.scale_log2, b1 = bf16_hi(rb) * p.scale_log2;
                                 qf[s][x] = pack_bf16(a0 * c0 - b0 * s0, a1 * c1 - b1 * s1);
                                 qf[s + 4][x] = pack_bf16(b0 * c0 + a0 * s0, b1 * c1 + a1 * s1);
                             }

@@ -100,10 +100,10 @@ static_assert(sizeof(PairTileInfo) == 80, "tile info layout");
 constexpr uint32_t TM_Q = 0, TM_S = 128, TM_O = 384;
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays below 2^8 between rescales
-// One pair of scores in kPolyEvery takes its exponentials on the FMA pipe (exp2_poly2), the
-// rest on the SFU: the SFU's 16 exponentials per clock per SM would otherwise take as long as
-// the tensor core's MMAs on the same tile.
-constexpr int kPolyEvery = 4;
+// kPolyOf8 pairs of scores in every 8 take their exponentials on the FMA pipe (exp2_poly2),
+// the rest on the SFU: with every exponential on the SFU the softmax of a tile takes longer
+// than the tensor core's MMAs on it (measured on B200: about 11.5 cycles per warp-wide ex2).
+constexpr int kPolyOf8 = 4;
 
 // Register split (launch: 384 threads x 168 registers): the loader/MMA warpgroup gives up
 // registers to the softmax (the whole 128-score row lives in registers) and the rotations.
@@ -136,9 +136,13 @@ __device__ __forceinline__ uint32_t map_rank(const void *p, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
     return r;
 }
-// Arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA).
+// Arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA).  The
+// data these arrivals publish lives in tensor memory and is ordered by tcgen05 fences around
+// the synchronisation, so the arrive keeps the default CTA-scope release: a cluster-scope
+// release measured about 870 cycles on B200 (against 8 for a local arrive), on the softmax's
+// critical path once per tile.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 __device__ __forceinline__ bool try_wait_cluster(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
@@ -677,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_pair_kernel(const __grid_
                 float x0 = f(2 * e), x1 = f(2 * e + 1);
                 add2(x0, x1, nmo, nmo);
                 float p0, p1;
-                if (e % kPolyEvery == kPolyEvery - 1) {
+                if (e % 8 >= 8 - kPolyOf8) {
                     exp2_poly2(x0, x1, p0, p1);
                 } else {
                     p0 = fast_exp2(x0);
