@@ -66,7 +66,7 @@ TRAFFIC = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
     #     -k regex:decode_split -s 3 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu --no-compare --no-e2e
     "decode_8b": {"sha": "c5296f2fb7ad0da4", "bytes": 785284352 + 8163072},
-    # the same with -k regex:prefill_pair
+    # the same with -k regex:prefill_tc
     "prefill_8b": {"sha": "", "bytes": 0},
 }
 
@@ -559,7 +559,7 @@ def run_prefill(args, world, peaks, peak_src, flush):
         "algorithmic_flops_per_launch": flops,
         "roofline": {"bound": "tensor", "kernel": "lazy_prefill_attn", "achieved": round(achieved, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_source": peak_src,
-                     "traffic": traffic_for("prefill_8b", "prefill_pair.cu")},
+                     "traffic": traffic_for("prefill_8b", "prefill_tc.cu")},
         **({"comparison": comparison} if comparison else {}),
     }
 

@@ -208,7 +208,7 @@ int prefill_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t 
     const long long units = static_cast<long long>(p.pf_mtiles) * p.hkv * num_req;
     if (units > (1LL << 30)) return LAZY_ERANGE;
     if (dry) return LAZY_OK;
-    int nsplit = prefill_split_units(units, prefill_wave_units(sm_count()));
+    int nsplit = prefill_split_units(units, sm_count());
     if (!workspace || ws_bytes < prefill_split_bytes(nsplit)) nsplit = 0;
     p.pf_nsplit = nsplit;
     p.pf_base = static_cast<int>(units) - nsplit;
@@ -216,13 +216,13 @@ int prefill_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t 
     p.ws_ml = nsplit ? p.ws_acc + static_cast<size_t>(nsplit) * 2 * kPrefillRows * 128 : nullptr;
     p.k_rows = static_cast<int>(k_rows);
     p.v_rows = static_cast<int>(static_cast<int64_t>(num_blocks) * p.hkv * 16);
-    CUtensorMap tk, tv, tk4, tv8;
+    CUtensorMap tk, tv, tk8, tv8;
     if (!make_rows_map(&tk, k_src, k_rows) || !make_rows_map(&tv, v_pool, p.v_rows)) return LAZY_ECUDA;
-    if (!make_blocks_map(&tk4, k_src, k_rows / (16 * p.hkv), p.hkv, 4) ||
+    if (!make_blocks_map(&tk8, k_src, k_rows / (16 * p.hkv), p.hkv, 8) ||
         !make_blocks_map(&tv8, v_pool, num_blocks, p.hkv, 8))
         return LAZY_ECUDA;
     // each request writes exactly its own query tokens' rows
-    return launch_rc(launch_prefill_pair(tk, tv, tk4, tv8, p, plain, static_cast<cudaStream_t>(stream)));
+    return launch_rc(launch_prefill_tc(tk, tv, tk8, tv8, p, plain, static_cast<cudaStream_t>(stream)));
 }
 
 // The side stream of lazy_mixed_attn and its fork/join events, one set per device, created at
@@ -331,8 +331,7 @@ size_t lazy_prefill_workspace_bytes(const lazy_attn_cfg *cfg, int num_req, int t
     if (!cfg || check_cfg(cfg) != LAZY_OK || num_req <= 0 || max_q <= 0) return 0;
     const int G = cfg->num_q_heads / cfg->num_kv_heads;
     const long long mtiles = (static_cast<long long>(max_q) * G + kPrefillRows - 1) / kPrefillRows;
-    return prefill_split_bytes(
-        prefill_split_units(mtiles * cfg->num_kv_heads * num_req, prefill_wave_units(sm_count())));
+    return prefill_split_bytes(prefill_split_units(mtiles * cfg->num_kv_heads * num_req, sm_count()));
 }
 
 int lazy_prefill_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *cu_q, const int32_t *q_pos0,

@@ -179,41 +179,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     return d;
 }
 
-// (a0, a1) -= (b0, b1)
-__device__ __forceinline__ void sub2(float &a0, float &a1, float b0, float b1) {
-    asm("{\n .reg .b64 x, y;\n mov.b64 x, {%0, %1};\n mov.b64 y, {%2, %3};\n sub.rn.f32x2 x, x, y;\n"
-        " mov.b64 {%0, %1}, x;\n}"
-        : "+f"(a0), "+f"(a1)
-        : "f"(b0), "f"(b1));
-}
-
-// 2^x for two arguments on the FMA pipe instead of the SFU, for x in [-120, 64]
-// (smaller arguments are raised to -120, whose power of two is below 2^-119).
-// x = n + f with n = round(x) taken from the low mantissa bits of x + 1.5 * 2^23 and
-// f in [-1/2, 1/2]; 2^f is the cubic of least maximum relative error on that interval
-// (coefficients from a Remez exchange, relative error <= 7.5e-5), and 2^n is added
-// to its exponent field.  Used for a share of a softmax row's exponentials, whose
-// results are rounded to bf16 (relative 2^-9) anyway.
-constexpr float kExp2C0 = 0.99992807f, kExp2C1 = 0.69326099f, kExp2C2 = 0.24261112f, kExp2C3 = 0.05517167f;
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float &y0, float &y1) {
-    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-    x0 = fmaxf(x0, -120.f);
-    x1 = fmaxf(x1, -120.f);
-    float t0 = x0, t1 = x1;
-    add2(t0, t1, kRound, kRound);        // round(x) in the low mantissa bits
-    float n0 = t0, n1 = t1;
-    sub2(n0, n1, kRound, kRound);        // round(x), exactly
-    float f0 = x0, f1 = x1;
-    sub2(f0, f1, n0, n1);                // f = x - round(x), exactly
-    float p0, p1;
-    fma2v(p0, p1, f0, f1, kExp2C3, kExp2C3, kExp2C2, kExp2C2);
-    fma2v(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
-    fma2v(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
-    // exponent field + round(x): (t_bits << 23) keeps exactly round(x) << 23 (mod 2^32)
-    y0 = __uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(p0));
-    y1 = __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(p1));
-}
-
 // 2^x via the SFU (PTX ex2.approx, relative error about 2^-22); 2^-inf = 0.
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;

@@ -89,11 +89,7 @@ cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const At
 // tk8, tv8: the same memory as (d, token, head, block) (one box = half of 8 consecutive blocks).
 cudaError_t launch_prefill_tc(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8,
                               const CUtensorMap &tv8, const AttnParams &p, bool plain, cudaStream_t s);
-// tk, tv: as above; tk4: the K source as (d, token, head, block) with a box of half of 4
-// consecutive blocks; tv8: the V pool with a box of half of 8 consecutive blocks.
-cudaError_t launch_prefill_pair(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk4,
-                                const CUtensorMap &tv8, const AttnParams &p, bool plain, cudaStream_t s);
-constexpr int kPrefillRows = 256;   // query rows per prefill work unit
+constexpr int kPrefillRows = 256;   // query rows per prefill CTA
 // Units of the last, partial wave that are split in two when that wave is at most half full
 // (one prefill CTA per SM): the grid then ends with two half-length CTAs per such unit.
 inline int prefill_split_units(long long units, int sms) {
@@ -101,8 +97,6 @@ inline int prefill_split_units(long long units, int sms) {
     const long long rem = units % sms;
     return (rem > 0 && 2 * rem <= sms) ? static_cast<int>(rem) : 0;
 }
-// Work units that run at once: one per pair of SMs (each unit is a cluster of two CTAs).
-inline int prefill_wave_units(int sms) { return sms / 2; }
 inline size_t prefill_split_bytes(int nsplit) {
     return static_cast<size_t>(nsplit) * 2 * kPrefillRows * (128 + 2) * sizeof(float);
 }
