@@ -63,11 +63,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Each figure holds for the kernel source whose hash it carries; a source edit voids it, except an
 # edit of comments alone (same lines), after which the hash is re-pinned.
 TRAFFIC = {
-    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
-    #     -k regex:decode_split -s 3 -c 1 python bench.py --steps 2 --warmup 3 --no-cpu --no-compare --no-e2e
-    "decode_8b": {"sha": "c5296f2fb7ad0da4", "bytes": 785284352 + 8163072},
-    # the same with -k regex:prefill_tc
-    "prefill_8b": {"sha": "", "bytes": 0},
+    # ncu --clock-control none --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
+    #     -k regex:decode_split -s 3 -c 1
+    #     python bench.py --steps 2 --warmup 3 --no-cpu --no-compare --no-e2e --no-distinct
+    "decode_8b": {"sha": "545dbebd3d15d2f3", "bytes": 786657024 + 6874112},
+    # the same command with --no-prefill --workload decode_8b_distinct
+    "decode_8b_distinct": {"sha": "545dbebd3d15d2f3", "bytes": 1095635456 + 7873024},
+    # the first command with -k regex:prefill_tc
+    "prefill_8b": {"sha": "196b11b5ee72ba24", "bytes": 301056000 + 26041344},
 }
 
 
