@@ -32,8 +32,8 @@
 //               blocks are consecutive in the pool, else two 2 KiB boxes per
 //               block
 //   warp 1      V producer: the same for V tiles, 2 stages
-//   warps 2, 3  MMA issuers for row tiles 0 and 1 (warp 2 also owns tensor
-//               memory): QK_t(j) then PV_t(j)
+//   warp 2      MMA issuer for both row tiles, in ping-pong order (and owner of
+//               tensor memory); warp 3 has no role
 //   warps 4-7   row tile 0, one thread per row: first the rotated query rows
 //               of the tile, then per K tile the online softmax with the whole
 //               128-column score row in registers (one tensor-memory load,
@@ -90,9 +90,9 @@ static_assert(kTcSmem <= 232448, "shared memory budget");
 static_assert(sizeof(TileInfo) == 80, "tile info layout");
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays below 2^8 between rescales
-// consumers of one tile-info entry: 8 softmax warps, the V producer, the two MMA warps, and
-// on the lazy path the 4 rotation warps
-constexpr int kInfoConsumers = 11;
+// consumers of one tile-info entry: 8 softmax warps, the V producer, the MMA warp, and on the
+// lazy path the 4 rotation warps
+constexpr int kInfoConsumers = 10;
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -183,12 +183,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     if (threadIdx.x == 0) {
         for (int i = 0; i < kKStages; ++i) {
             mbar_init(&bars[B_KFULL + i], 1);
-            mbar_init(&bars[B_KEMPTY + i], 2);
+            mbar_init(&bars[B_KEMPTY + i], 1);
             mbar_init(&bars[B_KROT + i], 4);
         }
         for (int i = 0; i < kVStages; ++i) {
             mbar_init(&bars[B_VFULL + i], 1);
-            mbar_init(&bars[B_VEMPTY + i], 2);
+            mbar_init(&bars[B_VEMPTY + i], 1);
         }
         for (int i = 0; i < kInfoStages; ++i) {
             mbar_init(&bars[B_IFULL + i], 1);
@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             mbar_init(&bars[B_ODONE + t], 1);
         }
         mbar_init(&bars[B_QFULL], 8);
-        mbar_init(&bars[B_DRAIN], 2);
+        mbar_init(&bars[B_DRAIN], 1);
         *abort_flag = 0;
         if (mt == 0 && kvh == 0 && n_words > p.max_words) set_status(p.d_status, LAZY_DSTATUS_BAD_TABLE);
         fence_barrier_init();
@@ -336,59 +336,104 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             for (int j = max(0, issued - kVStages); j < issued; ++j)
                 mbar_wait(&bars[B_VFULL + j % kVStages], (j / kVStages) & 1);
         }
-    } else if (warp == 2 || warp == 3) {
-        // ============================================================ MMA issuers
-        // Warp 2 issues row tile 0's MMAs, warp 3 row tile 1's: two independent
-        // issuers keep more MMAs in flight than one (measured on B200: about 86
-        // instead of about 100 cycles per 128x128x16 MMA).  Per tile the order
-        // is QK_t(j), then PV_t(j) once softmax t has written P_t(j); QK_t(j+1)
-        // follows PV_t(j) in issue order, which is what lets P_t live in S_t.
-        if (lane == 0) {
-            const int t = warp - 2;
-            const uint32_t idq = tc::idesc_bf16(128, 128, false);
-            const uint32_t idv = tc::idesc_bf16(128, 128, true);
-            const uint32_t sQ = smem_u32(sm + kOffQ), sK = smem_u32(sm + kOffK), sV = smem_u32(sm + kOffV);
-            const uint32_t tS = tbase + 128 * t, tO = tbase + 256 + 128 * t;
-            // descriptors at offset 0 of each buffer; a byte offset b is added as b >> 4
-            // to the start-address field (no carry: shared addresses are below 2^18)
-            const uint64_t dQ = tc::smem_desc(sQ + t * kTileBytes, 16, 1024), dK0 = tc::smem_desc(sK, 16, 1024);
-            const uint64_t dV0 = tc::smem_desc(sV, kHalfPlane, 1024);
-            bool ok = wait_or_abort(&bars[B_QFULL], 0, abort_flag, p.d_status);
-            for (int w = wbeg, j = 0; w < wend && ok; ++j) {
-                const int is = j % kInfoStages;
-                if (!wait_or_abort(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) break;
-                const int n = info[is].n;
-                mbar_arrive(&bars[B_IEMPTY + is]);
-                const int ks = j % kKStages;
-                // the plain path uses keys as loaded; the lazy path waits for their rotation
-                uint64_t *kready = ROTK ? &bars[B_KROT + ks] : &bars[B_KFULL + ks];
-                if (!wait_or_abort(kready, (j / kKStages) & 1, abort_flag, p.d_status)) break;
+    } else if (warp == 2) {
+        // ============================================================ MMA issuer
+        // One elected lane issues both row tiles' MMAs in the order
+        //   QK_0(0) QK_1(0) | PV_0(0) QK_0(1) | PV_1(0) QK_1(1) | PV_0(1) QK_0(2) | ...
+        // The tensor core runs them in issue order, so it works on one row tile
+        // while the other tile's softmax runs: softmax 0 of tile j+1 overlaps
+        // PV_1(j) QK_1(j+1), softmax 1 overlaps PV_0(j+1) QK_0(j+2).  (Two issuers,
+        // one per row tile, let the tensor core interleave both tiles' MMAs, which
+        // keeps the two softmaxes in step and the tensor core idle while they run.)
+        // QK_t(j+1) follows PV_t(j) in issue order, which is what lets P_t live in S_t.
+        // The whole warp runs the loop and waits; only the MMAs, commits and
+        // arrivals are issued by the elected lane, so the loop state stays uniform.
+        const uint32_t idq = tc::idesc_bf16(128, 128, false);
+        const uint32_t idv = tc::idesc_bf16(128, 128, true);
+        const uint32_t sQ = smem_u32(sm + kOffQ), sK = smem_u32(sm + kOffK), sV = smem_u32(sm + kOffV);
+        // descriptors at offset 0 of each buffer; a byte offset b is added as b >> 4
+        // to the start-address field (no carry: shared addresses are below 2^18)
+        const uint64_t dQ = tc::smem_desc(sQ, 16, 1024), dK0 = tc::smem_desc(sK, 16, 1024);
+        const uint64_t dV0 = tc::smem_desc(sV, kHalfPlane, 1024);
+        const bool leader = tc::elect_one();
+        bool ok = warp_wait(&bars[B_QFULL], 0, abort_flag, p.d_status);
+        int n = 0, j = 0;
+        for (int w = wbeg; ok && w < wend; ++j) {
+            // tile j's block count, from the tile-information ring (tile 0's read here,
+            // later tiles' one iteration ahead)
+            if (j == 0) {
+                if (!warp_wait(&bars[B_IFULL], 0, abort_flag, p.d_status)) break;
+                n = info[0].n;
+                __syncwarp();
+                if (leader) mbar_arrive(&bars[B_IEMPTY]);
+                if (!warp_wait(ROTK ? &bars[B_KROT] : &bars[B_KFULL], 0, abort_flag, p.d_status)) break;
                 tc::fence_after_sync();
-                const uint64_t kb = dK0 + static_cast<uint64_t>((ks * kTileBytes) >> 4);
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t o = static_cast<uint64_t>(((kk >> 2) * kHalfPlane + (kk & 3) * 32) >> 4);
-                    tc::mma_ss(tS, dQ + o, kb + o, idq, kk > 0 ? 1u : 0u);
+                    for (int t = 0; t < 2; ++t) {
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t o = static_cast<uint64_t>(((kk >> 2) * kHalfPlane + (kk & 3) * 32) >> 4);
+                            tc::mma_ss(tbase + 128 * t, dQ + static_cast<uint64_t>((t * kTileBytes) >> 4) + o, dK0 + o,
+                                       idq, kk > 0 ? 1u : 0u);
+                        }
+                        tc::commit(&bars[B_SFULL + t]);
+                    }
+                    tc::commit(&bars[B_KEMPTY]);
                 }
-                tc::commit(&bars[B_SFULL + t]);
-                tc::commit(&bars[B_KEMPTY + ks]);
-                // O_t += P_t V(j); P_t occupies the first 64 columns of S_t
-                const int vs = j % kVStages;
-                if (!wait_or_abort(&bars[B_VFULL + vs], (j / kVStages) & 1, abort_flag, p.d_status)) break;
-                if (!wait_or_abort(&bars[B_PFULL + t], j & 1, abort_flag, p.d_status)) break;
-                tc::fence_after_sync();
-                const uint64_t vb = dV0 + static_cast<uint64_t>((vs * kTileBytes) >> 4);
-                for (int k = 0; k < n; ++k)
-                    tc::mma_ts(tO, tS + 8 * k, vb + static_cast<uint64_t>((k * kBoxBytes) >> 4), idv,
-                               (j > 0 || k > 0) ? 1u : 0u);
-                tc::commit(&bars[B_ODONE + t]);
-                tc::commit(&bars[B_VEMPTY + vs]);
-                w += n;
+                __syncwarp();
             }
-            // every MMA this thread issued has completed before tensor memory is freed
-            tc::commit(&bars[B_DRAIN]);
-            mbar_wait(&bars[B_DRAIN], 0);
+            const bool next = w + n < wend;
+            int n_next = 0;
+            const int jn = j + 1, ksn = jn % kKStages;
+            if (next) {
+                const int is = jn % kInfoStages;
+                if (!warp_wait(&bars[B_IFULL + is], (jn / kInfoStages) & 1, abort_flag, p.d_status)) break;
+                n_next = info[is].n;
+                __syncwarp();
+                if (leader) mbar_arrive(&bars[B_IEMPTY + is]);
+                // the plain path uses keys as loaded; the lazy path waits for their rotation
+                if (!warp_wait(ROTK ? &bars[B_KROT + ksn] : &bars[B_KFULL + ksn], (jn / kKStages) & 1, abort_flag,
+                               p.d_status))
+                    break;
+            }
+            const int vs = j % kVStages;
+            if (!warp_wait(&bars[B_VFULL + vs], (j / kVStages) & 1, abort_flag, p.d_status)) break;
+            const uint64_t vb = dV0 + static_cast<uint64_t>((vs * kTileBytes) >> 4);
+            const uint64_t kb = dK0 + static_cast<uint64_t>((ksn * kTileBytes) >> 4);
+#pragma unroll 1
+            for (int t = 0; t < 2; ++t) {
+                if (!warp_wait(&bars[B_PFULL + t], j & 1, abort_flag, p.d_status)) { ok = false; break; }
+                tc::fence_after_sync();
+                if (leader) {
+                    // O_t += P_t V(j); P_t occupies the first 64 columns of S_t
+                    for (int k = 0; k < n; ++k)
+                        tc::mma_ts(tbase + 256 + 128 * t, tbase + 128 * t + 8 * k,
+                                   vb + static_cast<uint64_t>((k * kBoxBytes) >> 4), idv, (j > 0 || k > 0) ? 1u : 0u);
+                    tc::commit(&bars[B_ODONE + t]);
+                    if (t == 1) tc::commit(&bars[B_VEMPTY + vs]);
+                    if (next) {
+                        // S_t = Q'_t K(j+1)^T
+                        const uint64_t qb = dQ + static_cast<uint64_t>((t * kTileBytes) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t o = static_cast<uint64_t>(((kk >> 2) * kHalfPlane + (kk & 3) * 32) >> 4);
+                            tc::mma_ss(tbase + 128 * t, qb + o, kb + o, idq, kk > 0 ? 1u : 0u);
+                        }
+                        tc::commit(&bars[B_SFULL + t]);
+                        if (t == 1) tc::commit(&bars[B_KEMPTY + ksn]);
+                    }
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+            w += n;
+            n = n_next;
         }
+        // every MMA this warp issued has completed before tensor memory is freed
+        if (leader) tc::commit(&bars[B_DRAIN]);
+        __syncwarp();
+        mbar_wait(&bars[B_DRAIN], 0);
     }
     } else if (warp < 12) {
         // ============================================================ softmax (one row per thread)
