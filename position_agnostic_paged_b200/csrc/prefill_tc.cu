@@ -218,37 +218,40 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
     if (warp < 4) {
     setmaxnreg_dec<kProducerRegs>();
+    // The producers and the MMA issuer run their loops with the whole warp (control flow and
+    // loop state uniform); TMA copies, arrivals and MMAs are issued by an elected lane, or by
+    // lane k for block k of a tile whose blocks are not consecutive in the pool.
+    const bool leader = tc::elect_one();
     if (warp == 0) {
         // ============================================================ table walk + K producer
-        if (lane == 0) {
-            tma_prefetch_desc(&tmK);
-            int issued = 0;
-            for (int w = wbeg, j = 0; w < wend; ++j) {
-                // the tile: up to 8 consecutive words that share one offset
-                uint32_t wd[kTileBlocks];
+        if (leader) tma_prefetch_desc(&tmK);
+        int issued = 0;
+        for (int w = wbeg, j = 0; w < wend; ++j) {
+            // the tile: up to 8 consecutive words that share one offset
+            uint32_t wd[kTileBlocks];
 #pragma unroll
-                for (int k = 0; k < kTileBlocks; ++k) wd[k] = (w + k < wend) ? tbl[w + k] : 0xFFFFFFFFu;
-                const int off = word_offset(wd[0]);
-                int n = 1;
+            for (int k = 0; k < kTileBlocks; ++k) wd[k] = (w + k < wend) ? tbl[w + k] : 0xFFFFFFFFu;
+            const int off = word_offset(wd[0]);
+            int n = 1;
 #pragma unroll
-                for (int k = 1; k < kTileBlocks; ++k)
-                    if (n == k && w + k < wend && word_offset(wd[k]) == off) n = k + 1;
-                const int wn = w + n;
-                uint32_t mt_k[kTileBlocks];
-                bool full = n == kTileBlocks;
+            for (int k = 1; k < kTileBlocks; ++k)
+                if (n == k && w + k < wend && word_offset(wd[k]) == off) n = k + 1;
+            const int wn = w + n;
+            uint32_t mt_k[kTileBlocks];
+            bool full = n == kTileBlocks;
 #pragma unroll
-                for (int k = 0; k < kTileBlocks; ++k) {
-                    const uint32_t b = word_block(wd[k]);
-                    const bool ok = k < n && b < static_cast<uint32_t>(p.num_blocks);
-                    mt_k[k] = ok ? p.blk_meta[b] : 0u;
-                    if (k < n && !ok) set_status(p.d_status, LAZY_DSTATUS_BAD_BLOCK);
-                    full = full && meta_valid(mt_k[k]) == kBlockTokens &&
-                           off + meta_j0(mt_k[k]) + kBlockTokens - 1 <= Pbase;
-                }
-                const int flags = full ? kFull : 0;
-                // publish the tile information
-                const int is = j % kInfoStages;
-                if (!wait_or_abort(&bars[B_IEMPTY + is], ((j / kInfoStages) & 1) ^ 1, abort_flag, p.d_status)) break;
+            for (int k = 0; k < kTileBlocks; ++k) {
+                const uint32_t b = word_block(wd[k]);
+                const bool ok = k < n && b < static_cast<uint32_t>(p.num_blocks);
+                mt_k[k] = ok ? p.blk_meta[b] : 0u;
+                if (leader && k < n && !ok) set_status(p.d_status, LAZY_DSTATUS_BAD_BLOCK);
+                full = full && meta_valid(mt_k[k]) == kBlockTokens && off + meta_j0(mt_k[k]) + kBlockTokens - 1 <= Pbase;
+            }
+            const int flags = full ? kFull : 0;
+            // publish the tile information
+            const int is = j % kInfoStages;
+            if (!warp_wait(&bars[B_IEMPTY + is], ((j / kInfoStages) & 1) ^ 1, abort_flag, p.d_status)) break;
+            if (leader) {
                 TileInfo &ti = info[is];
 #pragma unroll
                 for (int k = 0; k < kTileBlocks; ++k) {
@@ -259,83 +262,90 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 ti.off = off;
                 ti.flags = flags;
                 mbar_arrive(&bars[B_IFULL + is]);
-                // K tile
-                const int ks = j % kKStages;
-                if (!wait_or_abort(&bars[B_KEMPTY + ks], ((j / kKStages) & 1) ^ 1, abort_flag, p.d_status)) break;
-                uint8_t *kd = sm + kOffK + ks * kTileBytes;
-                // blocks consecutive in the source: two 16 KiB boxes instead of 2n small ones
-                bool contig = true;
+            }
+            // K tile
+            const int ks = j % kKStages;
+            if (!warp_wait(&bars[B_KEMPTY + ks], ((j / kKStages) & 1) ^ 1, abort_flag, p.d_status)) break;
+            uint8_t *kd = sm + kOffK + ks * kTileBytes;
+            // blocks consecutive in the source: two 16 KiB boxes instead of 2n small ones
+            bool contig = true;
 #pragma unroll
-                for (int k = 1; k < kTileBlocks; ++k)
-                    contig = contig && (k >= n || word_block(wd[k]) == word_block(wd[0]) + static_cast<uint32_t>(k));
-                contig = PLAIN || (contig && word_block(wd[0]) < static_cast<uint32_t>(p.num_blocks) &&
-                                   word_block(wd[0]) + static_cast<uint32_t>(n) <= static_cast<uint32_t>(p.num_blocks));
-                if (contig) {
+            for (int k = 1; k < kTileBlocks; ++k)
+                contig = contig && (k >= n || word_block(wd[k]) == word_block(wd[0]) + static_cast<uint32_t>(k));
+            contig = PLAIN || (contig && word_block(wd[0]) < static_cast<uint32_t>(p.num_blocks) &&
+                               word_block(wd[0]) + static_cast<uint32_t>(n) <= static_cast<uint32_t>(p.num_blocks));
+            if (contig) {
+                if (leader) {
                     mbar_arrive_expect_tx(&bars[B_KFULL + ks], 2 * kHalfPlane);
                     const int z = PLAIN ? wbase + w : static_cast<int>(word_block(wd[0]));
                     tma_load_4d(kd, &tmK8, 0, 0, kvh, z, &bars[B_KFULL + ks]);
                     tma_load_4d(kd + kHalfPlane, &tmK8, kHalfDim, 0, kvh, z, &bars[B_KFULL + ks]);
-                } else {
-                mbar_arrive_expect_tx(&bars[B_KFULL + ks], n * kBlockBytes);
-                for (int k = 0; k < n; ++k) {
-                    const uint32_t b = word_block(wd[k]);
-                    int row;
-                    if (b >= static_cast<uint32_t>(p.num_blocks)) {
-                        row = p.k_rows;   // fully out of bounds: the box is zero-filled
-                    } else {
-                        row = PLAIN ? ((wbase + w + k) * p.hkv + kvh) * kBlockTokens
-                                    : (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens;
-                    }
-                    tma_load_2d(kd + k * kBoxBytes, &tmK, 0, row, &bars[B_KFULL + ks]);
-                    tma_load_2d(kd + kHalfPlane + k * kBoxBytes, &tmK, kHalfDim, row, &bars[B_KFULL + ks]);
                 }
+            } else {
+                if (leader) mbar_arrive_expect_tx(&bars[B_KFULL + ks], n * kBlockBytes);
+                __syncwarp();
+                if (lane < n) {
+                    uint32_t b = wd[0];
+#pragma unroll
+                    for (int k = 1; k < kTileBlocks; ++k) b = lane == k ? wd[k] : b;
+                    b = word_block(b);
+                    // fully out of bounds: the box is zero-filled
+                    const int row = b >= static_cast<uint32_t>(p.num_blocks)
+                                        ? p.k_rows
+                                        : (PLAIN ? ((wbase + w + lane) * p.hkv + kvh) * kBlockTokens
+                                                 : (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens);
+                    tma_load_2d(kd + lane * kBoxBytes, &tmK, 0, row, &bars[B_KFULL + ks]);
+                    tma_load_2d(kd + kHalfPlane + lane * kBoxBytes, &tmK, kHalfDim, row, &bars[B_KFULL + ks]);
                 }
-                issued = j + 1;
-                w = wn;
             }
-            for (int j = max(0, issued - kKStages); j < issued; ++j)
-                mbar_wait(&bars[B_KFULL + j % kKStages], (j / kKStages) & 1);
+            __syncwarp();
+            issued = j + 1;
+            w = wn;
         }
+        for (int j = max(0, issued - kKStages); j < issued; ++j)
+            mbar_wait(&bars[B_KFULL + j % kKStages], (j / kKStages) & 1);
     } else if (warp == 1) {
         // ============================================================ V producer
-        if (lane == 0) {
-            tma_prefetch_desc(&tmV);
-            int issued = 0;
-            for (int w = wbeg, j = 0; w < wend; ++j) {
-                const int is = j % kInfoStages;
-                if (!wait_or_abort(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) break;
-                const int n = info[is].n;
-                uint32_t blk[kTileBlocks];
-#pragma unroll
-                for (int k = 0; k < kTileBlocks; ++k) blk[k] = info[is].blk[k];
-                mbar_arrive(&bars[B_IEMPTY + is]);
-                const int vs = j % kVStages;
-                if (!wait_or_abort(&bars[B_VEMPTY + vs], ((j / kVStages) & 1) ^ 1, abort_flag, p.d_status)) break;
-                uint8_t *vd = sm + kOffV + vs * kTileBytes;
-                bool contig = blk[0] < static_cast<uint32_t>(p.num_blocks) &&
-                              blk[0] + static_cast<uint32_t>(n) <= static_cast<uint32_t>(p.num_blocks);
-#pragma unroll
-                for (int k = 1; k < kTileBlocks; ++k) contig = contig && (k >= n || blk[k] == blk[0] + static_cast<uint32_t>(k));
-                if (contig) {
+        if (leader) tma_prefetch_desc(&tmV);
+        int issued = 0;
+        for (int w = wbeg, j = 0; w < wend; ++j) {
+            const int is = j % kInfoStages;
+            if (!warp_wait(&bars[B_IFULL + is], (j / kInfoStages) & 1, abort_flag, p.d_status)) break;
+            const int n = info[is].n;
+            // lane k < n: block k of the tile
+            const uint32_t blk_l = info[is].blk[lane & (kTileBlocks - 1)];
+            const uint32_t blk0 = info[is].blk[0];
+            bool contig = blk0 < static_cast<uint32_t>(p.num_blocks) &&
+                          blk0 + static_cast<uint32_t>(n) <= static_cast<uint32_t>(p.num_blocks);
+            contig = __all_sync(0xffffffffu, contig && (lane >= n || blk_l == blk0 + static_cast<uint32_t>(lane)));
+            __syncwarp();
+            if (leader) mbar_arrive(&bars[B_IEMPTY + is]);
+            const int vs = j % kVStages;
+            if (!warp_wait(&bars[B_VEMPTY + vs], ((j / kVStages) & 1) ^ 1, abort_flag, p.d_status)) break;
+            uint8_t *vd = sm + kOffV + vs * kTileBytes;
+            if (contig) {
+                if (leader) {
                     mbar_arrive_expect_tx(&bars[B_VFULL + vs], 2 * kHalfPlane);
-                    tma_load_4d(vd, &tmV8, 0, 0, kvh, static_cast<int>(blk[0]), &bars[B_VFULL + vs]);
-                    tma_load_4d(vd + kHalfPlane, &tmV8, kHalfDim, 0, kvh, static_cast<int>(blk[0]), &bars[B_VFULL + vs]);
-                } else {
-                mbar_arrive_expect_tx(&bars[B_VFULL + vs], n * kBlockBytes);
-                for (int k = 0; k < n; ++k) {
-                    const int row = blk[k] >= static_cast<uint32_t>(p.num_blocks)
+                    tma_load_4d(vd, &tmV8, 0, 0, kvh, static_cast<int>(blk0), &bars[B_VFULL + vs]);
+                    tma_load_4d(vd + kHalfPlane, &tmV8, kHalfDim, 0, kvh, static_cast<int>(blk0), &bars[B_VFULL + vs]);
+                }
+            } else {
+                if (leader) mbar_arrive_expect_tx(&bars[B_VFULL + vs], n * kBlockBytes);
+                __syncwarp();
+                if (lane < n) {
+                    const int row = blk_l >= static_cast<uint32_t>(p.num_blocks)
                                         ? p.v_rows
-                                        : (static_cast<int>(blk[k]) * p.hkv + kvh) * kBlockTokens;
-                    tma_load_2d(vd + k * kBoxBytes, &tmV, 0, row, &bars[B_VFULL + vs]);
-                    tma_load_2d(vd + kHalfPlane + k * kBoxBytes, &tmV, kHalfDim, row, &bars[B_VFULL + vs]);
+                                        : (static_cast<int>(blk_l) * p.hkv + kvh) * kBlockTokens;
+                    tma_load_2d(vd + lane * kBoxBytes, &tmV, 0, row, &bars[B_VFULL + vs]);
+                    tma_load_2d(vd + kHalfPlane + lane * kBoxBytes, &tmV, kHalfDim, row, &bars[B_VFULL + vs]);
                 }
-                }
-                issued = j + 1;
-                w += n;
             }
-            for (int j = max(0, issued - kVStages); j < issued; ++j)
-                mbar_wait(&bars[B_VFULL + j % kVStages], (j / kVStages) & 1);
+            __syncwarp();
+            issued = j + 1;
+            w += n;
         }
+        for (int j = max(0, issued - kVStages); j < issued; ++j)
+            mbar_wait(&bars[B_VFULL + j % kVStages], (j / kVStages) & 1);
     } else if (warp == 2) {
         // ============================================================ MMA issuer
         // One elected lane issues both row tiles' MMAs in the order
@@ -355,7 +365,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         // to the start-address field (no carry: shared addresses are below 2^18)
         const uint64_t dQ = tc::smem_desc(sQ, 16, 1024), dK0 = tc::smem_desc(sK, 16, 1024);
         const uint64_t dV0 = tc::smem_desc(sV, kHalfPlane, 1024);
-        const bool leader = tc::elect_one();
         bool ok = warp_wait(&bars[B_QFULL], 0, abort_flag, p.d_status);
         int n = 0, j = 0;
         for (int w = wbeg; ok && w < wend; ++j) {
