@@ -227,57 +227,45 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         if (leader) tma_prefetch_desc(&tmK);
         int issued = 0;
         for (int w = wbeg, j = 0; w < wend; ++j) {
-            // the tile: up to 8 consecutive words that share one offset
-            uint32_t wd[kTileBlocks];
-#pragma unroll
-            for (int k = 0; k < kTileBlocks; ++k) wd[k] = (w + k < wend) ? tbl[w + k] : 0xFFFFFFFFu;
-            const int off = word_offset(wd[0]);
-            int n = 1;
-#pragma unroll
-            for (int k = 1; k < kTileBlocks; ++k)
-                if (n == k && w + k < wend && word_offset(wd[k]) == off) n = k + 1;
-            const int wn = w + n;
-            uint32_t mt_k[kTileBlocks];
-            bool full = n == kTileBlocks;
-#pragma unroll
-            for (int k = 0; k < kTileBlocks; ++k) {
-                const uint32_t b = word_block(wd[k]);
-                const bool ok = k < n && b < static_cast<uint32_t>(p.num_blocks);
-                mt_k[k] = ok ? p.blk_meta[b] : 0u;
-                if (leader && k < n && !ok) set_status(p.d_status, LAZY_DSTATUS_BAD_BLOCK);
-                full = full && meta_valid(mt_k[k]) == kBlockTokens && off + meta_j0(mt_k[k]) + kBlockTokens - 1 <= Pbase;
-            }
-            const int flags = full ? kFull : 0;
+            // the tile: up to 8 consecutive words that share one offset; lane k < 8 holds word k
+            const uint32_t wl = (lane < kTileBlocks && w + lane < wend) ? tbl[w + lane] : 0xFFFFFFFFu;
+            const int off = word_offset(__shfl_sync(0xffffffffu, wl, 0));
+            const bool same = lane < kTileBlocks && w + lane < wend && word_offset(wl) == off;
+            const int n = __ffs(~__ballot_sync(0xffffffffu, same)) - 1;   // lanes 0..n-1 share the offset
+            const uint32_t b = word_block(wl);
+            const bool inb = lane < n && b < static_cast<uint32_t>(p.num_blocks);
+            const uint32_t mt = inb ? p.blk_meta[b] : 0u;
+            if (lane < n && !inb) set_status(p.d_status, LAZY_DSTATUS_BAD_BLOCK);
+            const bool full = n == kTileBlocks &&
+                              __all_sync(0xffffffffu, lane >= n || (meta_valid(mt) == kBlockTokens &&
+                                                                    off + meta_j0(mt) + kBlockTokens - 1 <= Pbase));
+            // blocks consecutive in the source: two 16 KiB boxes instead of 2n small ones
+            const uint32_t b0 = __shfl_sync(0xffffffffu, b, 0);
+            const bool contig =
+                PLAIN || __all_sync(0xffffffffu, lane >= n || (inb && b == b0 + static_cast<uint32_t>(lane)));
             // publish the tile information
             const int is = j % kInfoStages;
             if (!warp_wait(&bars[B_IEMPTY + is], ((j / kInfoStages) & 1) ^ 1, abort_flag, p.d_status)) break;
+            TileInfo &ti = info[is];
+            if (lane < kTileBlocks) {
+                ti.blk[lane] = lane < n ? b : 0u;
+                ti.meta[lane] = mt;
+            }
             if (leader) {
-                TileInfo &ti = info[is];
-#pragma unroll
-                for (int k = 0; k < kTileBlocks; ++k) {
-                    ti.blk[k] = k < n ? word_block(wd[k]) : 0u;
-                    ti.meta[k] = mt_k[k];
-                }
                 ti.n = n;
                 ti.off = off;
-                ti.flags = flags;
-                mbar_arrive(&bars[B_IFULL + is]);
+                ti.flags = full ? kFull : 0;
             }
+            __syncwarp();
+            if (leader) mbar_arrive(&bars[B_IFULL + is]);
             // K tile
             const int ks = j % kKStages;
             if (!warp_wait(&bars[B_KEMPTY + ks], ((j / kKStages) & 1) ^ 1, abort_flag, p.d_status)) break;
             uint8_t *kd = sm + kOffK + ks * kTileBytes;
-            // blocks consecutive in the source: two 16 KiB boxes instead of 2n small ones
-            bool contig = true;
-#pragma unroll
-            for (int k = 1; k < kTileBlocks; ++k)
-                contig = contig && (k >= n || word_block(wd[k]) == word_block(wd[0]) + static_cast<uint32_t>(k));
-            contig = PLAIN || (contig && word_block(wd[0]) < static_cast<uint32_t>(p.num_blocks) &&
-                               word_block(wd[0]) + static_cast<uint32_t>(n) <= static_cast<uint32_t>(p.num_blocks));
             if (contig) {
                 if (leader) {
                     mbar_arrive_expect_tx(&bars[B_KFULL + ks], 2 * kHalfPlane);
-                    const int z = PLAIN ? wbase + w : static_cast<int>(word_block(wd[0]));
+                    const int z = PLAIN ? wbase + w : static_cast<int>(b0);
                     tma_load_4d(kd, &tmK8, 0, 0, kvh, z, &bars[B_KFULL + ks]);
                     tma_load_4d(kd + kHalfPlane, &tmK8, kHalfDim, 0, kvh, z, &bars[B_KFULL + ks]);
                 }
@@ -285,22 +273,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 if (leader) mbar_arrive_expect_tx(&bars[B_KFULL + ks], n * kBlockBytes);
                 __syncwarp();
                 if (lane < n) {
-                    uint32_t b = wd[0];
-#pragma unroll
-                    for (int k = 1; k < kTileBlocks; ++k) b = lane == k ? wd[k] : b;
-                    b = word_block(b);
                     // fully out of bounds: the box is zero-filled
-                    const int row = b >= static_cast<uint32_t>(p.num_blocks)
-                                        ? p.k_rows
-                                        : (PLAIN ? ((wbase + w + lane) * p.hkv + kvh) * kBlockTokens
-                                                 : (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens);
+                    const int row = !inb ? p.k_rows
+                                         : (PLAIN ? ((wbase + w + lane) * p.hkv + kvh) * kBlockTokens
+                                                  : (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens);
                     tma_load_2d(kd + lane * kBoxBytes, &tmK, 0, row, &bars[B_KFULL + ks]);
                     tma_load_2d(kd + kHalfPlane + lane * kBoxBytes, &tmK, kHalfDim, row, &bars[B_KFULL + ks]);
                 }
             }
             __syncwarp();
             issued = j + 1;
-            w = wn;
+            w += n;
         }
         for (int j = max(0, issued - kKStages); j < issued; ++j)
             mbar_wait(&bars[B_KFULL + j % kKStages], (j / kKStages) & 1);
@@ -545,13 +528,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             const TileInfo &ti = info[is];
             const int n = ti.n;
             const bool full = (ti.flags & kFull) != 0;
-            // visible keys of each 16-key block for this row: slots si < lim[k]
-            int lim[kTileBlocks];
+            // visible keys of each 16-key block for this row: slots si < lim_k (0..16), five bits
+            // per block in one 64-bit word
+            uint64_t limp = 0;
             float bk[kTileBlocks];   // ALiBi: bias of slot 0 of block k, slope * (o + j0 - p); 0 otherwise
 #pragma unroll
             for (int k = 0; k < kTileBlocks; ++k) {
                 const int nv = k < n ? meta_valid(ti.meta[k]) : 0;
-                lim[k] = max(0, min(nv, prow - ti.off - meta_j0(ti.meta[k]) + 1));
+                limp |= static_cast<uint64_t>(max(0, min(nv, prow - ti.off - meta_j0(ti.meta[k]) + 1))) << (5 * k);
                 bk[k] = ALIBI ? slope * static_cast<float>(ti.off + meta_j0(ti.meta[k]) - prow) : 0.f;
             }
             __syncwarp();
@@ -578,8 +562,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             }
             if (!full) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    sv[c] = (c & 15) < lim[c >> 4] ? sv[c] : 0xFF800000u;   // -inf: P = 0
+                for (int k = 0; k < kTileBlocks; ++k) {
+                    const int lim = static_cast<int>((limp >> (5 * k)) & 31u);
+#pragma unroll
+                    for (int c = 16 * k; c < 16 * k + 16; ++c)
+                        sv[c] = (c & 15) < lim ? sv[c] : 0xFF800000u;   // -inf: P = 0
+                }
             }
             // row max with three-input maxima (exact, so the order does not matter)
             auto f = [&](int c) { return __uint_as_float(sv[c]); };
