@@ -38,13 +38,14 @@ EncodeTiledFn encode_fn() {
 }
 
 // A pool (or materialised copy) viewed as rows of 128 bf16 (256 B); boxes of
-// 16 rows x 64 elements with the 128-byte swizzle (one half of a 16-token block).
-bool make_rows_map(CUtensorMap *map, const void *base, int64_t rows) {
+// box_rows rows x 64 elements with the 128-byte swizzle (by default one half of a
+// 16-token block).
+bool make_rows_map(CUtensorMap *map, const void *base, int64_t rows, int box_rows = 16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn || rows <= 0) return false;
     cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {256};
-    cuuint32_t box[2] = {64, 16};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -214,15 +215,26 @@ int prefill_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t 
     p.pf_base = static_cast<int>(units) - nsplit;
     p.ws_acc = static_cast<float *>(workspace);
     p.ws_ml = nsplit ? p.ws_acc + static_cast<size_t>(nsplit) * 2 * kPrefillRows * 128 : nullptr;
+    // with room after the split partials (16-byte aligned, as TMA requires), the query tiles
+    // are rotated by a first kernel and loaded by TMA; otherwise each CTA rotates its own
+    const size_t qoff = prefill_qprep_offset(nsplit);
+    if (workspace && ws_bytes >= qoff + prefill_qprep_bytes(units) && units * kPrefillRows <= INT32_MAX &&
+        (reinterpret_cast<uintptr_t>(workspace) + qoff) % 16 == 0)
+        p.q_prep = reinterpret_cast<uint16_t *>(static_cast<char *>(workspace) + qoff);
     p.k_rows = static_cast<int>(k_rows);
     p.v_rows = static_cast<int>(static_cast<int64_t>(num_blocks) * p.hkv * 16);
-    CUtensorMap tk, tv, tk8, tv8;
+    CUtensorMap tk, tv, tk8, tv8, tq;
     if (!make_rows_map(&tk, k_src, k_rows) || !make_rows_map(&tv, v_pool, p.v_rows)) return LAZY_ECUDA;
     if (!make_blocks_map(&tk8, k_src, k_rows / (16 * p.hkv), p.hkv, 8) ||
         !make_blocks_map(&tv8, v_pool, num_blocks, p.hkv, 8))
         return LAZY_ECUDA;
+    if (p.q_prep) {
+        if (!make_rows_map(&tq, p.q_prep, units * kPrefillRows, 128)) return LAZY_ECUDA;
+    } else {
+        tq = tk;   // not read
+    }
     // each request writes exactly its own query tokens' rows
-    return launch_rc(launch_prefill_tc(tk, tv, tk8, tv8, p, plain, static_cast<cudaStream_t>(stream)));
+    return launch_rc(launch_prefill_tc(tk, tv, tk8, tv8, tq, p, plain, static_cast<cudaStream_t>(stream)));
 }
 
 // The side stream of lazy_mixed_attn and its fork/join events, one set per device, created at
@@ -331,7 +343,8 @@ size_t lazy_prefill_workspace_bytes(const lazy_attn_cfg *cfg, int num_req, int t
     if (!cfg || check_cfg(cfg) != LAZY_OK || num_req <= 0 || max_q <= 0) return 0;
     const int G = cfg->num_q_heads / cfg->num_kv_heads;
     const long long mtiles = (static_cast<long long>(max_q) * G + kPrefillRows - 1) / kPrefillRows;
-    return prefill_split_bytes(prefill_split_units(mtiles * cfg->num_kv_heads * num_req, sm_count()));
+    const long long units = mtiles * cfg->num_kv_heads * num_req;
+    return prefill_qprep_offset(prefill_split_units(units, sm_count())) + prefill_qprep_bytes(units);
 }
 
 int lazy_prefill_attn(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *cu_q, const int32_t *q_pos0,

@@ -56,6 +56,7 @@ struct AttnParams {
     uint16_t *out;
     float *ws_acc;               // decode: [B][Hkv][S][G][128]
     float *ws_ml;                // decode: [B][Hkv][S][G][2]
+    uint16_t *q_prep;            // prefill: rotated query tiles [units][256][128] bf16, or null
     int *d_status;
     int num_req, hq, hkv, group, num_blocks, max_words;
     int words_per_split, n_splits;   // decode
@@ -86,9 +87,11 @@ cudaError_t launch_debug_bounded_wait(uint32_t polls, int complete, int *result,
 cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, bool plain,
                           cudaStream_t s);
 // tk, tv: the K source and V pool as rows of 128 bf16 (one box = half of one block);
-// tk8, tv8: the same memory as (d, token, head, block) (one box = half of 8 consecutive blocks).
+// tk8, tv8: the same memory as (d, token, head, block) (one box = half of 8 consecutive blocks);
+// tq: p.q_prep as rows of 128 bf16 (one box = half of 128 rows), used when p.q_prep is set.
 cudaError_t launch_prefill_tc(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8,
-                              const CUtensorMap &tv8, const AttnParams &p, bool plain, cudaStream_t s);
+                              const CUtensorMap &tv8, const CUtensorMap &tq, const AttnParams &p, bool plain,
+                              cudaStream_t s);
 constexpr int kPrefillRows = 256;   // query rows per prefill CTA
 // Units of the last, partial wave that are split in two when that wave is at most half full
 // (one prefill CTA per SM): the grid then ends with two half-length CTAs per such unit.
@@ -99,6 +102,11 @@ inline int prefill_split_units(long long units, int sms) {
 }
 inline size_t prefill_split_bytes(int nsplit) {
     return static_cast<size_t>(nsplit) * 2 * kPrefillRows * (128 + 2) * sizeof(float);
+}
+// The prepared query tiles follow the split partials in the workspace, 1 KiB aligned.
+inline size_t prefill_qprep_offset(int nsplit) { return (prefill_split_bytes(nsplit) + 1023) / 1024 * 1024; }
+inline size_t prefill_qprep_bytes(long long units) {
+    return static_cast<size_t>(units) * kPrefillRows * 128 * sizeof(uint16_t);
 }
 
 }  // namespace lazy

@@ -143,6 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                                                                  const __grid_constant__ CUtensorMap tmV,
                                                                  const __grid_constant__ CUtensorMap tmK8,
                                                                  const __grid_constant__ CUtensorMap tmV8,
+                                                                 const __grid_constant__ CUtensorMap tmQ,
                                                                  const AttnParams p) {
     constexpr bool PLAIN = MODE == kPlain;   // K source indexed by table position
     constexpr bool ROTK = MODE == kLazy;     // K tiles rotated in shared memory
@@ -199,7 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             mbar_init(&bars[B_PFULL + t], 4);
             mbar_init(&bars[B_ODONE + t], 1);
         }
-        mbar_init(&bars[B_QFULL], 8);
+        // the query tiles: written by the 8 softmax warps, or loaded prepared by one TMA arrival
+        mbar_init(&bars[B_QFULL], p.q_prep ? 1 : 8);
         mbar_init(&bars[B_DRAIN], 1);
         *abort_flag = 0;
         if (mt == 0 && kvh == 0 && n_words > p.max_words) set_status(p.d_status, LAZY_DSTATUS_BAD_TABLE);
@@ -426,6 +428,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         if (leader) tc::commit(&bars[B_DRAIN]);
         __syncwarp();
         mbar_wait(&bars[B_DRAIN], 0);
+    } else if (p.q_prep) {
+        // ============================================================ prepared query tiles
+        // Rows unit * 256 .. + 255 of the prepared query buffer (rotated and scaled by
+        // prefill_qprep_kernel): two row tiles, each two 64-column halves of 128 rows.
+        if (leader) {
+            tma_prefetch_desc(&tmQ);
+            mbar_arrive_expect_tx(&bars[B_QFULL], 2 * kTileBytes);
+            const int y = unit * kRows;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                tma_load_2d(sm + kOffQ + t * kTileBytes, &tmQ, 0, y + kTileRows * t, &bars[B_QFULL]);
+                tma_load_2d(sm + kOffQ + t * kTileBytes + kHalfPlane, &tmQ, kHalfDim, y + kTileRows * t, &bars[B_QFULL]);
+            }
+        }
+        __syncwarp();
+        // the loads land before the kernel's tensor memory is freed (the MMAs that read them
+        // have completed by then anyway); a wait that runs out only reports
+        mbar_wait(&bars[B_QFULL], 0);
     }
     } else if (warp < 12) {
         // ============================================================ softmax (one row per thread)
@@ -441,11 +461,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const int prow = pos0 + tok;
         const float slope = ALIBI ? slope_s[g] : 0.f;
         const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-        // Q'_i = R(p_i - P0) q_i for this warpgroup's row tile (R(p_i) on the plain path):
+        // Q'_i = R(p_i - P0) q_i for this warpgroup's row tile (R(p_i) on the plain path),
+        // unless the tiles arrive prepared by TMA:
         // thread (ch, rb) writes pairs 8ch..8ch+7 of rows rb + 16k; between rows rb + 16k and
         // rb + 16(k+1) the token advances by dlo = 16 / G or dlo + 1, so the angles advance by
         // rotations from two step tables.
-        {
+        if (!p.q_prep) {
             const int ch = row & 7, rb = row >> 3;
             const int dlo = 16 / G;
             float cA[8], sA[8], cB[8], sB[8];
@@ -794,14 +815,86 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(const AttnParams p
     reinterpret_cast<uint2 *>(p.out + (static_cast<size_t>(q0 + tok) * p.hq + kvh * G + g) * kHeadDim)[lane] = u;
 }
 
+// The query tiles of every work unit, rotated and scaled, ahead of the attention kernel:
+// row R of unit (m-tile mt, KV head kvh, request r) -- token R / G, head kvh * G + R % G --
+// becomes Q'_R = scale_log2 * R(p - qref) q at buffer row unit * 256 + R % 256, with
+// qref = P0 = q_pos0[r] + (256 mt) / G, the unit's first query position (0 on the plain path:
+// rotation to the absolute position).  Rows past the request's tokens are zero.  One thread
+// per (request, row, group of 8 rotation pairs); the angles of its 8 pairs are evaluated once
+// and applied to the row of every KV head.
+__global__ void __launch_bounds__(256) prefill_qprep_kernel(const AttnParams p, int plain) {
+    const int r = blockIdx.y;
+    const int R = blockIdx.x * 32 + (threadIdx.x >> 3), ch = threadIdx.x & 7;
+    const int G = p.group;
+    const int q0 = p.cu_q[r], T = p.cu_q[r + 1] - q0;
+    const int mt = R / kRows;
+    if (mt >= p.pf_mtiles || mt * kRows >= T * G) return;   // no unit of this request holds row R
+    const size_t dst_row0 = (static_cast<size_t>(r) * p.hkv * p.pf_mtiles + mt) * kRows + R % kRows;
+    const size_t unit_stride = static_cast<size_t>(p.pf_mtiles) * kRows;   // next KV head, same m-tile
+    if (R >= T * G) {
+        for (int kvh = 0; kvh < p.hkv; ++kvh) {
+            uint4 *d = reinterpret_cast<uint4 *>(p.q_prep + (dst_row0 + kvh * unit_stride) * kHeadDim);
+            d[ch] = make_uint4(0, 0, 0, 0);
+            d[8 + ch] = make_uint4(0, 0, 0, 0);
+        }
+        return;
+    }
+    const int tok = R / G, g = R % G;
+    const int pos0 = p.q_pos0[r];
+    const int delta = plain ? pos0 + tok : tok - (mt * kRows) / G;
+    float c[8], sn[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) rope_cos_sin(delta, p.rope.theta[8 * ch + e], c[e], sn[e]);
+    const float sc = p.scale_log2;
+    // eight KV heads at a time: all loads issued before the first store
+    constexpr int kHeadsPerPass = 8;
+    for (int kb = 0; kb < p.hkv; kb += kHeadsPerPass) {
+        uint4 a8[kHeadsPerPass], b8[kHeadsPerPass];
+#pragma unroll
+        for (int u = 0; u < kHeadsPerPass; ++u) {
+            if (kb + u < p.hkv) {
+                const uint4 *q = reinterpret_cast<const uint4 *>(
+                    p.q_raw + (static_cast<size_t>(q0 + tok) * p.hq + (kb + u) * G + g) * kHeadDim);
+                a8[u] = __ldg(q + ch);
+                b8[u] = __ldg(q + 8 + ch);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kHeadsPerPass; ++u) {
+            if (kb + u >= p.hkv) break;
+            const uint32_t *aw = reinterpret_cast<const uint32_t *>(&a8[u]);
+            const uint32_t *bw = reinterpret_cast<const uint32_t *>(&b8[u]);
+            uint4 lo, hi;
+            uint32_t *lw = reinterpret_cast<uint32_t *>(&lo);
+            uint32_t *hw = reinterpret_cast<uint32_t *>(&hi);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float a0 = bf16_lo(aw[e]) * sc, a1 = bf16_hi(aw[e]) * sc;
+                const float b0 = bf16_lo(bw[e]) * sc, b1 = bf16_hi(bw[e]) * sc;
+                const float c0 = c[2 * e], s0 = sn[2 * e], c1 = c[2 * e + 1], s1 = sn[2 * e + 1];
+                lw[e] = pack_bf16(a0 * c0 - b0 * s0, a1 * c1 - b1 * s1);
+                hw[e] = pack_bf16(b0 * c0 + a0 * s0, b1 * c1 + a1 * s1);
+            }
+            uint4 *d = reinterpret_cast<uint4 *>(p.q_prep + (dst_row0 + (kb + u) * unit_stride) * kHeadDim);
+            d[ch] = lo;
+            d[8 + ch] = hi;
+        }
+    }
+}
+
 template <int MODE>
 cudaError_t launch_t(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8, const CUtensorMap &tv8,
-                     const AttnParams &p, cudaStream_t s) {
+                     const CUtensorMap &tq, const AttnParams &p, cudaStream_t s) {
     auto kern = prefill_tc_kernel<MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
     if (e != cudaSuccess) return e;
     static_assert(kRows == kPrefillRows, "rows per CTA");
-    kern<<<p.pf_base + 2 * p.pf_nsplit, kThreads, kTcSmem, s>>>(tk, tv, tk8, tv8, p);
+    if (p.q_prep) {
+        prefill_qprep_kernel<<<dim3(p.pf_mtiles * (kRows / 32), p.num_req), 256, 0, s>>>(p, MODE == kPlain);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<p.pf_base + 2 * p.pf_nsplit, kThreads, kTcSmem, s>>>(tk, tv, tk8, tv8, tq, p);
     e = cudaGetLastError();
     if (e != cudaSuccess || p.pf_nsplit == 0) return e;
     prefill_combine_kernel<<<dim3(p.pf_nsplit, kRows / 8), 256, 0, s>>>(p);
@@ -811,9 +904,10 @@ cudaError_t launch_t(const CUtensorMap &tk, const CUtensorMap &tv, const CUtenso
 }  // namespace
 
 cudaError_t launch_prefill_tc(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8,
-                              const CUtensorMap &tv8, const AttnParams &p, bool plain, cudaStream_t s) {
-    if (plain) return launch_t<kPlain>(tk, tv, tk8, tv8, p, s);
-    return p.alibi ? launch_t<kAlibi>(tk, tv, tk8, tv8, p, s) : launch_t<kLazy>(tk, tv, tk8, tv8, p, s);
+                              const CUtensorMap &tv8, const CUtensorMap &tq, const AttnParams &p, bool plain,
+                              cudaStream_t s) {
+    if (plain) return launch_t<kPlain>(tk, tv, tk8, tv8, tq, p, s);
+    return p.alibi ? launch_t<kAlibi>(tk, tv, tk8, tv8, tq, p, s) : launch_t<kLazy>(tk, tv, tk8, tv8, tq, p, s);
 }
 
 }  // namespace lazy

@@ -96,7 +96,8 @@ class DeviceCase:
 
     def prefill(self, plain: bool = False, split: bool = True):
         """split: pass the workspace lazy_prefill_workspace_bytes asks for, so that the units of
-        a partial last wave run as two halves merged by the combine kernel."""
+        a partial last wave run as two halves merged by the combine kernel and the query tiles
+        are rotated by the preparation kernel; without it each CTA rotates its own query rows."""
         c = self.case
         n = c.cu_q.size - 1
         q_pos0 = []

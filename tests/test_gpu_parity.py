@@ -196,7 +196,8 @@ def _adv_requests(decode: bool):
 @pytest.mark.parametrize("kind", ["decode", "prefill", "prefill_unsplit"])
 def test_adversarial_cases_all_group_sizes(kind, hq, hkv):
     """prefill: every unit runs as two halves merged by the combine kernel (small batches leave
-    most SMs idle); prefill_unsplit: no workspace, one CTA per unit."""
+    most SMs idle), query tiles rotated by the preparation kernel; prefill_unsplit: no
+    workspace, one CTA per unit, each rotating its own query rows."""
     case = make_case(100 + hq + hkv, hq=hq, hkv=hkv, d=128, requests=_adv_requests(kind == "decode"))
     dc = DeviceCase(case)
     ref = oracle.attend(**case.oracle_kwargs())
