@@ -111,7 +111,7 @@ float scale_log2(const lazy_attn_cfg *cfg) {
 int launch_rc(cudaError_t e) { return e == cudaSuccess ? LAZY_OK : LAZY_ECUDA; }
 
 size_t decode_ws(const lazy_attn_cfg *cfg, int num_req, int max_words) {
-    const DecodePlan pl = decode_plan(num_req, cfg->num_kv_heads, max_words);
+    const DecodePlan pl = decode_plan(num_req, cfg->num_kv_heads, max_words, cfg->num_q_heads / cfg->num_kv_heads);
     const size_t parts = static_cast<size_t>(num_req) * cfg->num_kv_heads * pl.n_splits *
                          (cfg->num_q_heads / cfg->num_kv_heads);
     return parts * (128 + 2) * sizeof(float);
@@ -165,7 +165,7 @@ int decode_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *
     const size_t need = decode_ws(cfg, num_req, max_words);
     if (!workspace || ws_bytes < need) return LAZY_EWORKSPACE;
     if (dry) return LAZY_OK;
-    const DecodePlan pl = decode_plan(num_req, cfg->num_kv_heads, max_words);
+    const DecodePlan pl = decode_plan(num_req, cfg->num_kv_heads, max_words, p.group);
     p.q_raw = q_raw;
     p.q_pos = q_pos;
     p.k_rows = static_cast<int>(k_rows);
@@ -175,11 +175,12 @@ int decode_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *
     const size_t parts = static_cast<size_t>(num_req) * p.hkv * pl.n_splits * p.group;
     p.ws_acc = static_cast<float *>(workspace);
     p.ws_ml = p.ws_acc + parts * 128;
-    CUtensorMap tk, tv;
-    if (!make_rows_map(&tk, k_src, k_rows) ||
-        !make_rows_map(&tv, v_pool, static_cast<int64_t>(num_blocks) * p.hkv * 16))
+    CUtensorMap tk, tv, tk8, tv8;
+    if (!make_rows_map(&tk, k_src, k_rows) || !make_rows_map(&tv, v_pool, p.v_rows)) return LAZY_ECUDA;
+    if (!make_blocks_map(&tk8, k_src, k_rows / (16 * p.hkv), p.hkv, 8) ||
+        !make_blocks_map(&tv8, v_pool, num_blocks, p.hkv, 8))
         return LAZY_ECUDA;
-    return launch_rc(launch_decode(tk, tv, p, plain, static_cast<cudaStream_t>(stream)));
+    return launch_rc(launch_decode(tk, tv, tk8, tv8, p, plain, static_cast<cudaStream_t>(stream)));
 }
 
 int prefill_impl(const lazy_attn_cfg *cfg, const uint16_t *q_raw, const int32_t *cu_q, const int32_t *q_pos0,

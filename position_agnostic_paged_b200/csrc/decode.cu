@@ -7,17 +7,17 @@
 // at a change of segment offset (a new document); the (block ID, offset)
 // metadata is decoded from one register; the kernel reads only K and V.
 //
-// Work decomposition.  One CTA per (split, KV head, request); a split is a
-// range of consecutive table words (16-token blocks).  Warp 4 is the TMA
-// producer: for each word it loads the K block and the V block (4 KiB each,
-// two 128-byte-swizzled boxes) into a ring of shared-memory stages.  Warps
-// 0-3 consume: the G query heads of the KV head form the N dimension of
-// m16n8k16 tensor-core MMAs (S^T = K q^T, then O^T += V^T P^T), so each K/V
-// byte is read from HBM once and feeds all G heads.  Warps split the words of
-// a stage ring round-robin when G <= 8, and split the heads in groups of 8
-// when G is 16 or 32.  Per-warp online-softmax states are merged in shared
-// memory; split partials (m, l, acc) go to the workspace and a second kernel
-// combines them (flash-decoding).
+// Work decomposition (G <= 8 query heads per KV head; more heads run on the
+// tensor-memory kernel of decode_tc.cu).  One CTA per (split, KV head,
+// request); a split is a range of consecutive table words (16-token blocks).
+// Warp 4 is the TMA producer: for each word it loads the K block and the V
+// block (4 KiB each, two 128-byte-swizzled boxes) into a ring of shared-memory
+// stages.  Warps 0-3 consume: the G query heads of the KV head form the N
+// dimension of m16n8k16 tensor-core MMAs (S^T = K q^T, then O^T += V^T P^T),
+// so each K/V byte is read from HBM once and feeds all G heads.  Warps split
+// the words of a stage ring round-robin.  Per-warp online-softmax states are
+// merged in shared memory; split partials (m, l, acc) go to the workspace and
+// a second kernel combines them (flash-decoding).
 //
 // ALiBi (p.alibi): the frequency table is zero, so the query "rotation" is the
 // identity and runs once; each score gets slope_h * (o + j - p) in log2 units,
@@ -349,235 +349,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_split_kernel(const _
     }
 }
 
-// Decode for many query heads per KV head (G > 8, e.g. MQA): the heads form the M dimension of
-// the m16n8k16 MMAs instead of N, so that one warp serves 16 heads with each K/V fragment it
-// loads (S = Q' K^T with 16 heads x 16 keys per word, then O += P V with P taken straight from
-// the score fragments).  MT 16-head tiles per KV head (1 for G <= 16, 2 for G <= 32); consumer
-// warp w takes head tile w % MT and the words i = w / MT (mod 4 / MT) of the split.  Each thread
-// holds the rows (heads) lane/4 and lane/4 + 8 of its tile: the raw query as bf16 pairs, the
-// rotated query fragments, 16 x 4 output accumulators and the two rows' softmax state.
-template <int MT, bool PLAIN, int kDecodeStages>
-__global__ void __launch_bounds__(kDecodeThreads, 3) decode_heads_kernel(const __grid_constant__ CUtensorMap tmK,
-                                                                      const __grid_constant__ CUtensorMap tmV,
-                                                                      const AttnParams p) {
-    constexpr int KW = 4 / MT;   // warps sharing the words of one head tile
-    static_assert(kDecodeStages % 4 == 0, "the stage ring must be a multiple of the consumer warps");
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *stages = align1024(smem_raw);
-    __shared__ uint64_t full_bar[kDecodeStages], empty_bar[kDecodeStages];
-    __shared__ uint32_t stage_word[kDecodeStages], stage_meta[kDecodeStages];
-    __shared__ double theta_s[kHalfDim];
-    __shared__ float slope_s[32];
-
-    const int split = blockIdx.x, kvh = blockIdx.y, r = blockIdx.z;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int G = p.group;
-    const int wbase = p.table_indptr[r];
-    const int n_words = p.table_indptr[r + 1] - wbase;
-    const int lo = split * p.words_per_split;
-    const int cnt = max(0, min(n_words, lo + p.words_per_split) - lo);
-    const int qpos = p.q_pos[r];
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kDecodeStages; ++s) {
-            mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], MT);
-        }
-        if (split == 0 && n_words > p.max_words) set_status(p.d_status, LAZY_DSTATUS_BAD_TABLE);
-        fence_barrier_init();
-    }
-    if (threadIdx.x < kHalfDim) theta_s[threadIdx.x] = p.rope.theta[threadIdx.x];
-    if (threadIdx.x < 32) slope_s[threadIdx.x] = (p.alibi && threadIdx.x < G) ? p.alibi_log2[kvh * G + threadIdx.x] : 0.f;
-    __syncthreads();
-
-    const int mt = warp % MT, kl = warp / MT;
-    const int c = lane & 3, gr = lane >> 2;
-    const int h0 = 16 * mt + gr, h1 = h0 + 8;   // heads (rows) of this thread in the group
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-    float oacc[16][4];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-
-    if (warp == 4) {
-        decode_producer<PLAIN, kDecodeStages>(tmK, tmV, p, stages, full_bar, empty_bar, stage_word, stage_meta,
-                                              kvh, wbase, lo, cnt, lane);
-    } else {
-        // raw query, A-fragment order: k-step s, register x: head (x & 1 ? h1 : h0), head-dim
-        // elements 16s + 8(x >> 1) + 2c and + 1
-        // raw query pairs of this thread, read from global memory (L1-resident after the first
-        // rotation) whenever the query is rotated, to keep registers for the accumulators
-        const uint16_t *qb = p.q_raw + (static_cast<size_t>(r) * p.hq + kvh * G) * kHeadDim;
-        auto qraw = [&](int s, int x) -> uint32_t {
-            const int h = (x & 1) ? h1 : h0;
-            return h < G ? __ldg(reinterpret_cast<const unsigned int *>(qb + h * kHeadDim + 16 * s + 8 * (x >> 1) + 2 * c))
-                         : 0u;
-        };
-        uint32_t qf[8][4];
-        int cur_off = INT_MIN;
-        const float sl0 = slope_s[h0 < 32 ? h0 : 0], sl1 = slope_s[h1 < 32 ? h1 : 0];
-        const uint32_t stage0 = smem_u32(stages);
-        const int mi = lane >> 3, li = lane & 7;
-        const int k_key = li + 8 * (mi >> 1), k_dc = 8 * (mi & 1);   // K rows as B fragments
-        const int v_key = li + 8 * (mi & 1), v_dc = 8 * (mi >> 1);   // V rows as B fragments (.trans)
-
-        for (int i = kl; i < cnt; i += KW) {
-            const int st = i % kDecodeStages;
-            const uint32_t ph = (i / kDecodeStages) & 1;
-            if (!mbar_wait(&full_bar[st], ph)) {
-                set_status(p.d_status, LAZY_DSTATUS_TIMEOUT);
-                break;
-            }
-            const uint32_t w = stage_word[st];
-            const uint32_t b = word_block(w);
-            if (b < static_cast<uint32_t>(p.num_blocks)) {
-                const uint32_t meta = stage_meta[st];
-                const int off = word_offset(w);
-                const int off_rot = PLAIN ? 0 : (p.alibi ? qpos : off);
-                if (off_rot != cur_off) {
-                    // Q' = R(q_pos - offset) q * scale: pairs (i, i + 64) sit in k-steps s and s + 4
-                    cur_off = off_rot;
-                    const int delta = qpos - off_rot;
-#pragma unroll
-                    for (int s = 0; s < 4; ++s)
-#pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            const int i0 = 16 * s + 8 * half + 2 * c;
-                            float c0, s0, c1, s1;
-                            rope_cos_sin(delta, theta_s[i0], c0, s0);
-                            rope_cos_sin(delta, theta_s[i0 + 1], c1, s1);
-#pragma unroll
-                            for (int hr = 0; hr < 2; ++hr) {
-                                const int x = 2 * half + hr;
-                                const uint32_t ra = qraw(s, x), rb = qraw(s + 4, x);
-                                const float a0 = bf16_lo(ra) * p.scale_log2, a1 = bf16_hi(ra) * p.scale_log2;
-                                const float b0 = bf16_lo(rb) * p.scale_log2, b1 = bf16_hi(rb) * p.scale_log2;
-                                qf[s][x] = pack_bf16(a0 * c0 - b0 * s0, a1 * c1 - b1 * s1);
-                                qf[s + 4][x] = pack_bf16(b0 * c0 + a0 * s0, b1 * c1 + a1 * s1);
-                            }
-                        }
-                }
-                const uint32_t kbase = stage0 + st * kStageBytes;
-                const uint32_t vbase = kbase + kBlockBytes;
-                // S[16 heads][16 keys] = Q' K^T: n-tiles of keys 0-7 and 8-15
-                float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(kbase + swz_offset(k_key, 16 * s + k_dc, kBlockTokens), b0, b1, b2, b3);
-                    mma_bf16(sacc[0], qf[s][0], qf[s][1], qf[s][2], qf[s][3], b0, b1);
-                    mma_bf16(sacc[1], qf[s][0], qf[s][1], qf[s][2], qf[s][3], b2, b3);
-                }
-                const int j0 = meta_j0(meta), nv = meta_valid(meta);
-                const int kpos = off + j0 - qpos;   // key position - query position, slot 0
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int kidx = 8 * nt + 2 * c + e;
-                        if (p.alibi) {
-                            sacc[nt][e] = fmaf(sl0, static_cast<float>(kpos + kidx), sacc[nt][e]);
-                            sacc[nt][2 + e] = fmaf(sl1, static_cast<float>(kpos + kidx), sacc[nt][2 + e]);
-                        }
-                        const bool vis = kidx < nv && kpos + kidx <= 0;
-                        if (!vis) sacc[nt][e] = sacc[nt][2 + e] = -INFINITY;
-                    }
-                // row maxima over the 16 keys: 4 per thread, then across the quad
-                float bm[2] = {max3(sacc[0][0], sacc[0][1], fmaxf(sacc[1][0], sacc[1][1])),
-                               max3(sacc[0][2], sacc[0][3], fmaxf(sacc[1][2], sacc[1][3]))};
-#pragma unroll
-                for (int x = 1; x < 4; x <<= 1) {
-                    bm[0] = fmaxf(bm[0], __shfl_xor_sync(0xffffffffu, bm[0], x));
-                    bm[1] = fmaxf(bm[1], __shfl_xor_sync(0xffffffffu, bm[1], x));
-                }
-                uint32_t pa[4];
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                    const float mn = fmaxf(m_run[hr], bm[hr]);
-                    const float mu = mn == -INFINITY ? 0.f : mn;
-                    if (mn != m_run[hr]) {
-                        const float sc = fast_exp2(m_run[hr] - mu);
-                        l_run[hr] *= sc;
-#pragma unroll
-                        for (int t = 0; t < 16; ++t) {
-                            oacc[t][2 * hr] *= sc;
-                            oacc[t][2 * hr + 1] *= sc;
-                        }
-                        m_run[hr] = mn;
-                    }
-                    float pr[4];
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) pr[2 * nt + e] = fast_exp2(sacc[nt][2 * hr + e] - mu);
-                    l_run[hr] += (pr[0] + pr[1]) + (pr[2] + pr[3]);
-                    // A fragment of P: (row hr, keys 2c..) then (row hr, keys 8 + 2c..)
-                    pa[hr] = pack_bf16(pr[0], pr[1]);
-                    pa[2 + hr] = pack_bf16(pr[2], pr[3]);
-                }
-                // O[16 heads][128] += P[16 heads][16 keys] V[16 keys][128]
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4_t(vbase + swz_offset(v_key, 16 * u + v_dc, kBlockTokens), b0, b1, b2, b3);
-                    mma_bf16(oacc[2 * u], pa[0], pa[1], pa[2], pa[3], b0, b1);
-                    mma_bf16(oacc[2 * u + 1], pa[0], pa[1], pa[2], pa[3], b2, b3);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty_bar[st]);
-        }
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr)
-#pragma unroll
-            for (int x = 1; x < 4; x <<= 1) l_run[hr] += __shfl_xor_sync(0xffffffffu, l_run[hr], x);
-    }
-    __syncthreads();   // every stage consumed, every copy landed: stage memory is free
-
-    // ---------------------------------------------------------------- merge warps, write split partial
-    constexpr int GP = 16 * MT;                                   // padded heads
-    float *sm_acc = reinterpret_cast<float *>(stages);           // [KW][GP][128]
-    float *sm_m = sm_acc + KW * GP * kHeadDim;                   // [KW][GP]
-    float *sm_l = sm_m + KW * GP;
-    if (warp < 4) {
-#pragma unroll
-        for (int t = 0; t < 16; ++t)
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const int h = (x >> 1) ? h1 : h0;
-                const int d = 8 * t + 2 * c + (x & 1);
-                sm_acc[(kl * GP + h) * kHeadDim + d] = oacc[t][x];
-            }
-        if (c == 0) {
-            sm_m[kl * GP + h0] = m_run[0];
-            sm_l[kl * GP + h0] = l_run[0];
-            sm_m[kl * GP + h1] = m_run[1];
-            sm_l[kl * GP + h1] = l_run[1];
-        }
-    }
-    __syncthreads();
-    const size_t part = (static_cast<size_t>(r) * p.hkv + kvh) * p.n_splits + split;
-    for (int it = threadIdx.x; it < G * kHeadDim; it += blockDim.x) {
-        const int g = it / kHeadDim, d = it % kHeadDim;
-        float M = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < KW; ++k) M = fmaxf(M, sm_m[k * GP + g]);
-        float L = 0.f, A = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int k = 0; k < KW; ++k) {
-                const float wgt = fast_exp2(sm_m[k * GP + g] - M);
-                L += wgt * sm_l[k * GP + g];
-                A += wgt * sm_acc[(k * GP + g) * kHeadDim + d];
-            }
-        }
-        p.ws_acc[(part * G + g) * kHeadDim + d] = A;
-        if (d == 0) {
-            p.ws_ml[(part * G + g) * 2 + 0] = M;
-            p.ws_ml[(part * G + g) * 2 + 1] = L;
-        }
-    }
-}
-
 // out[r][h][:] = sum_s acc_s 2^(m_s - M) / sum_s l_s 2^(m_s - M); zero if nothing was visible.
 __global__ void __launch_bounds__(128) decode_combine_kernel(const AttnParams p) {
     const int h = blockIdx.x % p.hq, r = blockIdx.x / p.hq;
@@ -620,46 +391,38 @@ cudaError_t launch_decode_nt(const CUtensorMap &tk, const CUtensorMap &tv, const
     return launch_decode_t<NT, PLAIN, kDefaultStages>(tk, tv, p, s);
 }
 
-template <int MT, bool PLAIN>
-cudaError_t launch_decode_heads(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, cudaStream_t s) {
-    auto kern = decode_heads_kernel<MT, PLAIN, kDefaultStages>;
-    const size_t smem = decode_smem(kDefaultStages);
-    static_assert(decode_smem(kDefaultStages) >= 1024 + size_t(4 / MT) * 16 * MT * (kHeadDim + 2) * 4, "merge area");
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid(p.n_splits, p.hkv, p.num_req);
-    kern<<<grid, kDecodeThreads, smem, s>>>(tk, tv, p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    decode_combine_kernel<<<p.num_req * p.hq, kHeadDim, 0, s>>>(p);
-    return cudaGetLastError();
-}
-
 }  // namespace
 
-DecodePlan decode_plan(int num_req, int hkv, int max_words) {
+DecodePlan decode_plan(int num_req, int hkv, int max_words, int group) {
     DecodePlan pl;
     const int units = max(1, num_req * hkv);
-    // aim at about 2000 CTAs (several waves over 148 SMs at ~3 resident CTAs
-    // each) while keeping at least 8 words (128 keys) per split
-    const int target = 2048;
+    const bool tc = group >= kDecodeTcMinGroup;
+    // warp-MMA kernels: about 2000 CTAs (several waves over 148 SMs at ~3 resident CTAs each),
+    // at least 8 words (128 keys) per split; tensor-memory kernel (one CTA per SM): about 600
+    // CTAs, at least 16 words (two key tiles) per split
+    const int target = tc ? 592 : 2048;
+    const int min_words = tc ? 16 : 8;
     int splits = (target + units - 1) / units;
-    const int max_splits = max(1, (max_words + 7) / 8);
+    const int max_splits = max(1, (max_words + min_words - 1) / min_words);
     splits = max(1, min(splits, max_splits));
     const int wps = max(1, (max_words + splits - 1) / splits);
     pl.words_per_split = wps;
-    pl.n_splits = max(1, (max_words + wps - 1) / wps);
+    pl.grid_splits = max(1, (max_words + wps - 1) / wps);
+    pl.n_splits = tc ? 2 * pl.grid_splits : pl.grid_splits;
     return pl;
 }
 
-cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, bool plain,
-                          cudaStream_t s) {
-    // G <= 8: heads as the N dimension (one warp's 8 heads share every K/V fragment);
-    // G > 8: heads as the M dimension, 16 per warp
-    if (p.group <= 8) return plain ? launch_decode_nt<1, true>(tk, tv, p, s) : launch_decode_nt<1, false>(tk, tv, p, s);
-    if (p.group <= 16)
-        return plain ? launch_decode_heads<1, true>(tk, tv, p, s) : launch_decode_heads<1, false>(tk, tv, p, s);
-    return plain ? launch_decode_heads<2, true>(tk, tv, p, s) : launch_decode_heads<2, false>(tk, tv, p, s);
+cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8,
+                          const CUtensorMap &tv8, const AttnParams &p, bool plain, cudaStream_t s) {
+    // G <= 8: heads as the N dimension of warp MMAs (one warp's 8 heads share every K/V
+    // fragment); more heads per KV head: heads as the rows of tcgen05 MMAs in tensor memory
+    if (p.group >= kDecodeTcMinGroup) return launch_decode_tc(tk, tv, tk8, tv8, p, plain, s);
+    return plain ? launch_decode_nt<1, true>(tk, tv, p, s) : launch_decode_nt<1, false>(tk, tv, p, s);
+}
+
+cudaError_t launch_decode_combine(const AttnParams &p, cudaStream_t s) {
+    decode_combine_kernel<<<p.num_req * p.hq, kHeadDim, 0, s>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace lazy

@@ -73,19 +73,29 @@ struct AttnParams {
     float alibi_log2[kMaxAlibiHeads];   // ALiBi slope of query head h, times log2(e)
 };
 
-// Decode split plan shared by the workspace query and the launch.
+// Decode split plan shared by the workspace query and the launch: CTAs per (request, KV head)
+// (grid_splits, each over words_per_split table words) and split partials per (request, KV
+// head) (n_splits: one per CTA, or two -- one per softmax stream -- for the tensor-memory
+// kernel used when a KV head serves more than 8 query heads).
 struct DecodePlan {
     int words_per_split;
+    int grid_splits;
     int n_splits;
 };
-DecodePlan decode_plan(int num_req, int hkv, int max_words);
+DecodePlan decode_plan(int num_req, int hkv, int max_words, int group);
+constexpr int kDecodeTcMinGroup = 9;   // query heads per KV head from which decode_tc runs
 
 cudaError_t launch_kv_write(const KvWriteParams &p, cudaStream_t s);
 cudaError_t launch_decode_table(const DecodeTableParams &p, cudaStream_t s);
 cudaError_t launch_materialize(const MaterializeParams &p, cudaStream_t s);
 cudaError_t launch_debug_bounded_wait(uint32_t polls, int complete, int *result, int *d_status, cudaStream_t s);
-cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &p, bool plain,
-                          cudaStream_t s);
+// tk8, tv8 as for the prefill (used by the tensor-memory kernel, G >= kDecodeTcMinGroup).
+cudaError_t launch_decode(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8,
+                          const CUtensorMap &tv8, const AttnParams &p, bool plain, cudaStream_t s);
+cudaError_t launch_decode_tc(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8,
+                             const CUtensorMap &tv8, const AttnParams &p, bool plain, cudaStream_t s);
+// Merges the p.n_splits partials of every (request, query head) into the output.
+cudaError_t launch_decode_combine(const AttnParams &p, cudaStream_t s);
 // tk, tv: the K source and V pool as rows of 128 bf16 (one box = half of one block);
 // tk8, tv8: the same memory as (d, token, head, block) (one box = half of 8 consecutive blocks);
 // tq: p.q_prep as rows of 128 bf16 (one box = half of 128 rows), used when p.q_prep is set.
