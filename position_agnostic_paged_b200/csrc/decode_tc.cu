@@ -24,11 +24,16 @@
 // own split partial and the combine kernel merges them with the other splits.
 //   warp 0   producer: walks the table one word per lane, publishes tile
 //            information, TMA-loads each tile's K and V into a stage
-//   warp 1   MMA issuer: QK(j) into S_{j%2}, then PV(j-1) from P_{(j-1)%2}
+//   warp 1   MMA issuer: QK(j) into S_{j%2} and PV(j-1) from P_{(j-1)%2}, in the
+//            order their inputs become ready
 //   warp 2   query rotation: Q' = R(q_pos - o) q * scale for each new segment
-//            offset o, into the single query buffer (rows = heads)
-//   warp 4   softmax of stream 0 (tensor-memory lanes 0-31 = heads)
-//   warp 8   softmax of stream 1
+//            offset o, computed ahead and stored into the single query buffer
+//            once the previous one is no longer read; the G heads are written
+//            twice, as rows 0..G-1 and 32..32+G-1
+//   warp 4   softmax of stream 0: tensor-memory lanes 0-31 (rows 0-31)
+//   warp 5   softmax of stream 1: lanes 32-63 (rows 32-63, the second copy of
+//            the heads), so that the two streams' softmaxes run on different
+//            sub-partitions of the SM
 // Tensor memory (512 columns): S0 [0,128) (P0 = its first 64 columns),
 // S1 [128,256) (P1), O0 [256,384), O1 [384,512).
 #include <climits>
@@ -45,7 +50,7 @@ constexpr int kTB = 8;                              // blocks per tile
 constexpr int kTileB = 128 * kHeadDim * 2;          // 32 KiB: 128 rows of 128 bf16
 constexpr int kHalfP = kTileB / 2;                  // 16 KiB: one 64-column half plane
 constexpr int kStages = 3, kInfo = 8;
-constexpr int kThreadsTc = 288;                     // 9 warps
+constexpr int kThreadsTc = 256;                     // 8 warps
 
 struct DInfo {
     uint32_t blk[kTB];
@@ -96,11 +101,11 @@ __device__ __forceinline__ bool wwait(uint64_t *bar, uint32_t parity, volatile i
 // at absolute positions, indexed by table position; query rotated once by q_pos), 2 ALiBi
 // (nothing rotated, bias slope_h * (key position - q_pos) added to each score).
 template <int MODE>
+// one CTA per SM (shared memory allows no more)
 __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
-                                                                  const __grid_constant__ CUtensorMap tmV,
-                                                                  const __grid_constant__ CUtensorMap tmK8,
-                                                                  const __grid_constant__ CUtensorMap tmV8,
-                                                                  const AttnParams p) {
+                                                  const __grid_constant__ CUtensorMap tmV,
+                                                  const __grid_constant__ CUtensorMap tmK8,
+                                                  const __grid_constant__ CUtensorMap tmV8, const AttnParams p) {
     constexpr bool PLAIN = MODE == 1;
     constexpr bool ALIBI = MODE == 2;
     extern __shared__ uint8_t smem_raw[];
@@ -239,72 +244,84 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
         const uint64_t dQ = tc::smem_desc(smem_u32(sm + kOffQ), 16, 1024);
         const uint64_t dK0 = tc::smem_desc(smem_u32(sm + kOffK), 16, 1024);
         const uint64_t dV0 = tc::smem_desc(smem_u32(sm + kOffV), kHalfP, 1024);
+        // Two actions are pending at a time: QK(j) (needs K/V tile j and, at a new offset, the new
+        // query) and PV(j-1) (needs P(j-1)); whichever is ready first is issued, QK(j) first when
+        // both are, so that neither waits behind the other's producer.
         int prev_n = 0, gen = -1, cur_rot = INT_MIN, j = 0;
-        bool ok = true;
-        for (int w = lo; w < hi; ++j) {
-            const int is = j % kInfo;
-            if (!wwait(&bars[B_IFULL + is], (j / kInfo) & 1, abort_flag, p.d_status)) { ok = false; break; }
-            const int n = info[is].n, off = info[is].off;
-            __syncwarp();
-            if (leader) mbar_arrive(&bars[B_IEMPTY + is]);
-            const int rot = PLAIN ? 0 : (ALIBI ? qpos : off);
-            if (rot != cur_rot) {
-                // the query for this offset: wait until the rotation warp has written it, after
-                // every MMA that read the previous one has completed
-                cur_rot = rot;
-                ++gen;
-                if (gen > 0 && leader) tc::commit(&bars[B_QFREE]);
+        bool ok = true, prev_tile = false;   // prev_tile: tile j-1 exists (and still needs its PV)
+        for (int w = lo; ok; ++j) {
+            const bool has_qk = w < hi;
+            int n = 0;
+            if (has_qk) {
+                const int is = j % kInfo;
+                if (!wwait(&bars[B_IFULL + is], (j / kInfo) & 1, abort_flag, p.d_status)) { ok = false; break; }
+                n = info[is].n;
+                const int off = info[is].off;
                 __syncwarp();
-                if (!wwait(&bars[B_QREADY], gen & 1, abort_flag, p.d_status)) { ok = false; break; }
+                if (leader) mbar_arrive(&bars[B_IEMPTY + is]);
+                const int rot = PLAIN ? 0 : (ALIBI ? qpos : off);
+                if (rot != cur_rot) {
+                    // every MMA that read the previous query has been issued (QK(j-1) at the latest)
+                    cur_rot = rot;
+                    ++gen;
+                    if (gen > 0 && leader) tc::commit(&bars[B_QFREE]);
+                    __syncwarp();
+                }
             }
+            const bool has_pv = prev_tile;
+            if (!has_qk && !has_pv) break;
+            bool need_qk = has_qk, need_pv = has_pv, need_q = has_qk;   // need_q: query not yet seen ready
             const int st = j % kStages, t = j & 1;
-            if (!wwait(&bars[B_KVFULL + st], (j / kStages) & 1, abort_flag, p.d_status)) { ok = false; break; }
-            tc::fence_after_sync();
-            if (leader) {
-                const uint64_t kb = dK0 + static_cast<uint64_t>((st * kTileB) >> 4);
+            const int u = (j - 1) & 1, su = (j + kStages - 1) % kStages;
+            uint32_t polls = 0;
+            while (need_qk || need_pv) {
+                if (need_qk) {
+                    if (need_q) need_q = !__all_sync(0xffffffffu, mbar_test_wait(&bars[B_QREADY], gen & 1));
+                    if (!need_q && __all_sync(0xffffffffu, mbar_test_wait(&bars[B_KVFULL + st], (j / kStages) & 1))) {
+                        tc::fence_after_sync();
+                        if (leader) {
+                            const uint64_t kb = dK0 + static_cast<uint64_t>((st * kTileB) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t o = static_cast<uint64_t>(((kk >> 2) * kHalfP + (kk & 3) * 32) >> 4);
-                    tc::mma_ss(tbase + 128 * t, dQ + o, kb + o, idq, kk > 0 ? 1u : 0u);
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint64_t o = static_cast<uint64_t>(((kk >> 2) * kHalfP + (kk & 3) * 32) >> 4);
+                                tc::mma_ss(tbase + 128 * t, dQ + o, kb + o, idq, kk > 0 ? 1u : 0u);
+                            }
+                            tc::commit(&bars[B_SFULL + t]);
+                        }
+                        __syncwarp();
+                        need_qk = false;
+                        continue;
+                    }
                 }
-                tc::commit(&bars[B_SFULL + t]);
-            }
-            __syncwarp();
-            if (j > 0) {
-                // PV(j-1): O_u += P_u V(j-1), u = (j-1) % 2, its P in the first 64 columns of S_u
-                const int u = (j - 1) & 1, su = (j - 1) % kStages;
-                if (!wwait(&bars[B_PFULL + u], ((j - 1) >> 1) & 1, abort_flag, p.d_status)) { ok = false; break; }
-                tc::fence_after_sync();
-                if (leader) {
-                    const uint64_t vb = dV0 + static_cast<uint64_t>((su * kTileB) >> 4);
-                    for (int k = 0; k < prev_n; ++k)
-                        tc::mma_ts(tbase + 256 + 128 * u, tbase + 128 * u + 8 * k,
-                                   vb + static_cast<uint64_t>((k * kBoxBytes) >> 4), idv,
-                                   (j - 1 > 1 || k > 0) ? 1u : 0u);
-                    tc::commit(&bars[B_ODONE + u]);
-                    tc::commit(&bars[B_KVEMPTY + su]);
+                if (need_pv && __all_sync(0xffffffffu, mbar_test_wait(&bars[B_PFULL + u], ((j - 1) >> 1) & 1))) {
+                    // PV(j-1): O_u += P_u V(j-1), P_u in the first 64 columns of S_u
+                    tc::fence_after_sync();
+                    if (leader) {
+                        const uint64_t vb = dV0 + static_cast<uint64_t>((su * kTileB) >> 4);
+                        for (int k = 0; k < prev_n; ++k)
+                            tc::mma_ts(tbase + 256 + 128 * u, tbase + 128 * u + 8 * k,
+                                       vb + static_cast<uint64_t>((k * kBoxBytes) >> 4), idv,
+                                       (j - 1 > 1 || k > 0) ? 1u : 0u);
+                        tc::commit(&bars[B_ODONE + u]);
+                        tc::commit(&bars[B_KVEMPTY + su]);
+                    }
+                    __syncwarp();
+                    need_pv = false;
+                    continue;
                 }
-                __syncwarp();
+                // nothing ready: bounded, like every other wait
+                if (++polls > (kWaitPolls << 2) || ((polls & 255) == 0 && *abort_flag)) {
+                    if (polls > (kWaitPolls << 2)) {
+                        *abort_flag = 1;
+                        if (leader) set_status(p.d_status, LAZY_DSTATUS_TIMEOUT);
+                    }
+                    ok = false;
+                    break;
+                }
             }
             prev_n = n;
+            prev_tile = has_qk;
             w += n;
-        }
-        if (ok && j > 0) {
-            // PV of the last tile
-            const int u = (j - 1) & 1, su = (j - 1) % kStages;
-            if (wwait(&bars[B_PFULL + u], ((j - 1) >> 1) & 1, abort_flag, p.d_status)) {
-                tc::fence_after_sync();
-                if (leader) {
-                    const uint64_t vb = dV0 + static_cast<uint64_t>((su * kTileB) >> 4);
-                    for (int k = 0; k < prev_n; ++k)
-                        tc::mma_ts(tbase + 256 + 128 * u, tbase + 128 * u + 8 * k,
-                                   vb + static_cast<uint64_t>((k * kBoxBytes) >> 4), idv,
-                                   (j - 1 > 1 || k > 0) ? 1u : 0u);
-                    tc::commit(&bars[B_ODONE + u]);
-                    tc::commit(&bars[B_KVEMPTY + su]);
-                }
-                __syncwarp();
-            }
         }
         // every MMA this warp issued has completed before tensor memory is freed
         if (leader) tc::commit(&bars[B_DRAIN]);
@@ -319,6 +336,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
         int gen = -1, cur_rot = INT_MIN;
         const uint4 *qrow =
             reinterpret_cast<const uint4 *>(p.q_raw + (static_cast<size_t>(r) * p.hq + kvh * G + lane) * kHeadDim);
+        const float sc = p.scale_log2;
         for (int w = lo, j = 0; w < hi; ++j) {
             const int is = j % kInfo;
             if (!wwait(&bars[B_IFULL + is], (j / kInfo) & 1, abort_flag, p.d_status)) break;
@@ -330,26 +348,36 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
             if (rot == cur_rot) continue;
             cur_rot = rot;
             ++gen;
-            // the previous query is no longer read once every MMA issued before QFREE completed
-            if (gen > 0 && !wwait(&bars[B_QFREE], (gen - 1) & 1, abort_flag, p.d_status)) break;
+            // The new query is computed into registers as soon as its tile's information appears
+            // (up to the ring's depth ahead of the MMAs); only the store waits until the previous
+            // query is no longer read (every MMA issued before QFREE completed).
             const int delta = qpos - rot;
             float c0, s0, c1, s1;
             rope_cos_sin(delta, p.rope.theta[lane], c0, s0);
             rope_cos_sin(delta, p.rope.theta[lane + 32], c1, s1);
+            __syncwarp();   // the previous rotation's reads of the angle table are done
             cs[lane] = make_float2(c0, s0);
             cs[lane + 32] = make_float2(c1, s1);
             __syncwarp();
-            uint8_t *qd = sm + kOffQ;
-            const float sc = p.scale_log2;
+            uint4 lo8[8], hi8[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-                uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
-                if (lane < G) {
-                    const uint4 a4 = qrow[c], b4 = qrow[8 + c];   // elements 8c.. and 64 + 8c..
-                    const uint32_t *aw = reinterpret_cast<const uint32_t *>(&a4);
-                    const uint32_t *bw = reinterpret_cast<const uint32_t *>(&b4);
-                    uint32_t *lw = reinterpret_cast<uint32_t *>(&lo4);
-                    uint32_t *hw = reinterpret_cast<uint32_t *>(&hi4);
+                lo8[c] = make_uint4(0, 0, 0, 0);
+                hi8[c] = make_uint4(0, 0, 0, 0);
+            }
+            if (lane < G) {
+                uint4 a8[8], b8[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    a8[c] = __ldg(qrow + c);       // elements 8c .. 8c + 7
+                    b8[c] = __ldg(qrow + 8 + c);   // elements 64 + 8c ..
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t *aw = reinterpret_cast<const uint32_t *>(&a8[c]);
+                    const uint32_t *bw = reinterpret_cast<const uint32_t *>(&b8[c]);
+                    uint32_t *lw = reinterpret_cast<uint32_t *>(&lo8[c]);
+                    uint32_t *hw = reinterpret_cast<uint32_t *>(&hi8[c]);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 q0 = cs[8 * c + 2 * e], q1 = cs[8 * c + 2 * e + 1];
@@ -359,22 +387,32 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
                         hw[e] = pack_bf16(b0 * q0.x + a0 * q0.y, b1 * q1.x + a1 * q1.y);
                     }
                 }
+            }
+            if (gen > 0 && !wwait(&bars[B_QFREE], (gen - 1) & 1, abort_flag, p.d_status)) break;
+            uint8_t *qd = sm + kOffQ;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                // rows lane and 32 + lane (same swizzle phase: 32 is a multiple of 8)
                 const uint32_t soff = lane * 128 + ((c ^ (lane & 7)) << 4);
-                *reinterpret_cast<uint4 *>(qd + soff) = lo4;
-                *reinterpret_cast<uint4 *>(qd + kHalfP + soff) = hi4;
+                *reinterpret_cast<uint4 *>(qd + soff) = lo8[c];
+                *reinterpret_cast<uint4 *>(qd + kHalfP + soff) = hi8[c];
+                *reinterpret_cast<uint4 *>(qd + 32 * 128 + soff) = lo8[c];
+                *reinterpret_cast<uint4 *>(qd + kHalfP + 32 * 128 + soff) = hi8[c];
             }
             fence_proxy_async_smem();   // generic-proxy writes become visible to the tensor core
             __syncwarp();
             if (leader) mbar_arrive(&bars[B_QREADY]);
         }
-    } else if (warp == 4 || warp == 8) {
+    } else if (warp == 4 || warp == 5) {
         // ============================================================ softmax (one head per lane)
         // Stream t takes tiles j with j % 2 == t; every tile's information is read (to follow the
         // word ranges), only the stream's own tiles are processed.  The whole 128-column score
         // row of the lane's head is held in registers: one tensor-memory load, mask, max,
         // 2^(S - m), one store of P over the consumed S columns; O rescaled lazily.
-        const int t = warp == 4 ? 0 : 1;
-        const uint32_t tS = tbase + 128 * t, tO = tbase + 256 + 128 * t;   // lanes 0-31
+        const int t = warp - 4;
+        // stream t's rows 32t .. 32t + 31 = tensor-memory lanes of this warp's quarter
+        const uint32_t lane_off = static_cast<uint32_t>(32 * t) << 16;
+        const uint32_t tS = tbase + lane_off + 128 * t, tO = tbase + lane_off + 256 + 128 * t;
         const float slope = (ALIBI && lane < G) ? p.alibi_log2[kvh * G + lane] : 0.f;
         float m_run = -INFINITY, l_run = 0.f;
         int k = 0;   // tiles of this stream processed
