@@ -14,7 +14,7 @@
 // up with at HBM speed (their accumulators cap the CTAs per SM).  Here the
 // heads are the rows of 128 x 128 tcgen05 MMAs (rows G..127 are padding whose
 // results are never read), scores and the output accumulate in tensor memory,
-// and one CTA per SM streams 128-key tiles through a three-stage ring.
+// and one CTA per SM streams 128-key tiles through three-stage K and V rings.
 //
 // CTA = one split (a range of table words) of one KV head of one request.
 // Tiles are up to 8 consecutive words of one segment.  Two softmax streams
@@ -22,8 +22,10 @@
 // buffer S_t, output accumulator O_t and online-softmax state, so that one
 // stream's softmax overlaps the other stream's MMAs; each stream writes its
 // own split partial and the combine kernel merges them with the other splits.
-//   warp 0   producer: walks the table one word per lane, publishes tile
-//            information, TMA-loads each tile's K and V into a stage
+//   warp 0   K producer: walks the table one word per lane, publishes tile
+//            information, TMA-loads each tile's K into a ring of three stages
+//   warp 3   V producer (and owner of tensor memory): each tile's V into a ring
+//            of its own, so that a V stage held until PV does not hold back K
 //   warp 1   MMA issuer: QK(j) into S_{j%2} and PV(j-1) from P_{(j-1)%2}, in the
 //            order their inputs become ready
 //   warp 2   query rotation: Q' = R(q_pos - o) q * scale for each new segment
@@ -68,7 +70,8 @@ constexpr int kOffK = kOffQ + kTileB;
 constexpr int kOffV = kOffK + kStages * kTileB;
 constexpr int kOffInfo = kOffV + kStages * kTileB;
 constexpr int kOffBar = kOffInfo + kInfo * static_cast<int>(sizeof(DInfo));
-constexpr int B_KVFULL = 0, B_KVEMPTY = B_KVFULL + kStages, B_IFULL = B_KVEMPTY + kStages,
+constexpr int B_KFULL = 0, B_KEMPTY = B_KFULL + kStages, B_VFULL = B_KEMPTY + kStages,
+              B_VEMPTY = B_VFULL + kStages, B_IFULL = B_VEMPTY + kStages,
               B_IEMPTY = B_IFULL + kInfo, B_SFULL = B_IEMPTY + kInfo, B_PFULL = B_SFULL + 2,
               B_ODONE = B_PFULL + 2, B_QREADY = B_ODONE + 2, B_QFREE = B_QREADY + 1, B_DRAIN = B_QFREE + 1,
               kBars = B_DRAIN + 1;
@@ -77,8 +80,9 @@ constexpr int kOffMisc = kOffCs + kHalfDim * 8;     // tensor-memory address, ab
 constexpr int kSmemUse = kOffMisc + 16;
 constexpr size_t kSmemTc = kSmemUse + 1024;
 static_assert(kSmemTc <= 232448, "shared memory budget");
-// consumers of a tile-information entry: the issuer, the rotation warp, both softmax warps
-constexpr int kInfoReaders = 4;
+// consumers of a tile-information entry: the V producer, the issuer, the rotation warp, both
+// softmax warps
+constexpr int kInfoReaders = 5;
 constexpr float kRescale = 8.0f;   // log2 units: P stays below 2^8 between rescales
 
 __device__ __forceinline__ uint8_t *align1k(uint8_t *p) {
@@ -128,8 +132,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&bars[B_KVFULL + i], 1);
-            mbar_init(&bars[B_KVEMPTY + i], 1);
+            mbar_init(&bars[B_KFULL + i], 1);
+            mbar_init(&bars[B_KEMPTY + i], 1);
+            mbar_init(&bars[B_VFULL + i], 1);
+            mbar_init(&bars[B_VEMPTY + i], 1);
         }
         for (int i = 0; i < kInfo; ++i) {
             mbar_init(&bars[B_IFULL + i], 1);
@@ -194,37 +200,26 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
             }
             __syncwarp();
             if (leader) mbar_arrive(&bars[B_IFULL + is]);
+            // K tile; its stage is free again once QK of the tile three back has completed
             const int st = j % kStages;
-            if (!wwait(&bars[B_KVEMPTY + st], ((j / kStages) & 1) ^ 1, abort_flag, p.d_status)) break;
+            if (!wwait(&bars[B_KEMPTY + st], ((j / kStages) & 1) ^ 1, abort_flag, p.d_status)) break;
             uint8_t *kd = sm + kOffK + st * kTileB;
-            uint8_t *vd = sm + kOffV + st * kTileB;
-            uint64_t *fb = &bars[B_KVFULL + st];
+            uint64_t *fb = &bars[B_KFULL + st];
             const bool k_contig = PLAIN || contig;   // the materialised copy is indexed by table position
             if (leader) {
-                mbar_arrive_expect_tx(fb, (k_contig ? 2 * kHalfP : n * kBlockBytes) + (contig ? 2 * kHalfP : n * kBlockBytes));
+                mbar_arrive_expect_tx(fb, k_contig ? 2 * kHalfP : n * kBlockBytes);
                 if (k_contig) {
                     const int z = PLAIN ? wbase + w : static_cast<int>(b0);
                     tma4d(kd, &tmK8, 0, 0, kvh, z, fb);
                     tma4d(kd + kHalfP, &tmK8, kHalfDim, 0, kvh, z, fb);
                 }
-                if (contig) {
-                    tma4d(vd, &tmV8, 0, 0, kvh, static_cast<int>(b0), fb);
-                    tma4d(vd + kHalfP, &tmV8, kHalfDim, 0, kvh, static_cast<int>(b0), fb);
-                }
             }
             __syncwarp();
-            if (lane < n) {
+            if (!k_contig && lane < n) {
                 // fully out of bounds: the box is zero-filled
-                if (!k_contig) {
-                    const int row = !inb ? p.k_rows : (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens;
-                    tma_load_2d(kd + lane * kBoxBytes, &tmK, 0, row, fb);
-                    tma_load_2d(kd + kHalfP + lane * kBoxBytes, &tmK, kHalfDim, row, fb);
-                }
-                if (!contig) {
-                    const int row = !inb ? p.v_rows : (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens;
-                    tma_load_2d(vd + lane * kBoxBytes, &tmV, 0, row, fb);
-                    tma_load_2d(vd + kHalfP + lane * kBoxBytes, &tmV, kHalfDim, row, fb);
-                }
+                const int row = !inb ? p.k_rows : (static_cast<int>(b) * p.hkv + kvh) * kBlockTokens;
+                tma_load_2d(kd + lane * kBoxBytes, &tmK, 0, row, fb);
+                tma_load_2d(kd + kHalfP + lane * kBoxBytes, &tmK, kHalfDim, row, fb);
             }
             __syncwarp();
             issued = j + 1;
@@ -232,7 +227,47 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
         }
         // every copy has landed before the kernel ends
         for (int j = max(0, issued - kStages); j < issued; ++j)
-            mbar_wait(&bars[B_KVFULL + j % kStages], (j / kStages) & 1);
+            mbar_wait(&bars[B_KFULL + j % kStages], (j / kStages) & 1);
+    } else if (warp == 3) {
+        // ============================================================ V producer
+        // V tiles in their own ring: a V stage is held from its load until PV of its tile, so
+        // loading it in step with K would tie the K loads to the much later PV.
+        if (leader) tma_prefetch_desc(&tmV);
+        int issued = 0;
+        for (int w = lo, j = 0; w < hi; ++j) {
+            const int is = j % kInfo;
+            if (!wwait(&bars[B_IFULL + is], (j / kInfo) & 1, abort_flag, p.d_status)) break;
+            const int n = info[is].n;
+            const uint32_t blk_l = info[is].blk[lane & (kTB - 1)];   // lane b < n: block b of the tile
+            const uint32_t blk0 = info[is].blk[0];
+            __syncwarp();
+            if (leader) mbar_arrive(&bars[B_IEMPTY + is]);
+            const bool inb = lane < n && blk_l < static_cast<uint32_t>(p.num_blocks);
+            const bool contig =
+                __all_sync(0xffffffffu, lane >= n || (inb && blk_l == blk0 + static_cast<uint32_t>(lane)));
+            const int st = j % kStages;
+            if (!wwait(&bars[B_VEMPTY + st], ((j / kStages) & 1) ^ 1, abort_flag, p.d_status)) break;
+            uint8_t *vd = sm + kOffV + st * kTileB;
+            uint64_t *fb = &bars[B_VFULL + st];
+            if (leader) {
+                mbar_arrive_expect_tx(fb, contig ? 2 * kHalfP : n * kBlockBytes);
+                if (contig) {
+                    tma4d(vd, &tmV8, 0, 0, kvh, static_cast<int>(blk0), fb);
+                    tma4d(vd + kHalfP, &tmV8, kHalfDim, 0, kvh, static_cast<int>(blk0), fb);
+                }
+            }
+            __syncwarp();
+            if (!contig && lane < n) {
+                const int row = !inb ? p.v_rows : (static_cast<int>(blk_l) * p.hkv + kvh) * kBlockTokens;
+                tma_load_2d(vd + lane * kBoxBytes, &tmV, 0, row, fb);
+                tma_load_2d(vd + kHalfP + lane * kBoxBytes, &tmV, kHalfDim, row, fb);
+            }
+            __syncwarp();
+            issued = j + 1;
+            w += n;
+        }
+        for (int j = max(0, issued - kStages); j < issued; ++j)
+            mbar_wait(&bars[B_VFULL + j % kStages], (j / kStages) & 1);
     } else if (warp == 1) {
         // ============================================================ MMA issuer
         // Order QK(0) | QK(1) PV(0) | QK(2) PV(1) | ...: S_t(j) (t = j % 2) is computed while the
@@ -277,7 +312,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
             while (need_qk || need_pv) {
                 if (need_qk) {
                     if (need_q) need_q = !__all_sync(0xffffffffu, mbar_test_wait(&bars[B_QREADY], gen & 1));
-                    if (!need_q && __all_sync(0xffffffffu, mbar_test_wait(&bars[B_KVFULL + st], (j / kStages) & 1))) {
+                    if (!need_q && __all_sync(0xffffffffu, mbar_test_wait(&bars[B_KFULL + st], (j / kStages) & 1))) {
                         tc::fence_after_sync();
                         if (leader) {
                             const uint64_t kb = dK0 + static_cast<uint64_t>((st * kTileB) >> 4);
@@ -287,13 +322,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
                                 tc::mma_ss(tbase + 128 * t, dQ + o, kb + o, idq, kk > 0 ? 1u : 0u);
                             }
                             tc::commit(&bars[B_SFULL + t]);
+                            tc::commit(&bars[B_KEMPTY + st]);
                         }
                         __syncwarp();
                         need_qk = false;
                         continue;
                     }
                 }
-                if (need_pv && __all_sync(0xffffffffu, mbar_test_wait(&bars[B_PFULL + u], ((j - 1) >> 1) & 1))) {
+                if (need_pv && __all_sync(0xffffffffu, mbar_test_wait(&bars[B_PFULL + u], ((j - 1) >> 1) & 1) &&
+                                                           mbar_test_wait(&bars[B_VFULL + su], ((j - 1) / kStages) & 1))) {
                     // PV(j-1): O_u += P_u V(j-1), P_u in the first 64 columns of S_u
                     tc::fence_after_sync();
                     if (leader) {
@@ -303,7 +340,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
                                        vb + static_cast<uint64_t>((k * kBoxBytes) >> 4), idv,
                                        (j - 1 > 1 || k > 0) ? 1u : 0u);
                         tc::commit(&bars[B_ODONE + u]);
-                        tc::commit(&bars[B_KVEMPTY + su]);
+                        tc::commit(&bars[B_VEMPTY + su]);
                     }
                     __syncwarp();
                     need_pv = false;
