@@ -255,12 +255,13 @@ typedef struct lazy_decode_batch {
  * and lazy_decode_attn(decode) (the same kernels on the same inputs); the
  * difference is scheduling.  Both batches are validated on the host before
  * anything is enqueued, so an error leaves nothing half-launched.  The
- * prefill runs on `stream`; the decode runs on a side stream of the library
- * (one per device, created at the first call, non-blocking), forked from
- * `stream` before the prefill and joined back into it after the decode, so
- * work enqueued on `stream` afterwards sees both outputs.  Launched after the
- * prefill, the decode's CTAs take the SMs that the prefill's last wave
- * leaves idle, and no launch gap separates the two kernels.  Either batch
+ * prefill runs on a side stream of the library (one per device, created at
+ * the first call, non-blocking, with the device's highest stream priority),
+ * forked from `stream` and joined back into it after the decode; the decode
+ * runs on `stream` once the prefill's attention kernel is enqueued, so work
+ * enqueued on `stream` afterwards sees both outputs.  With the higher
+ * priority the prefill's CTAs are dispatched first, and the decode's CTAs
+ * take the SMs that the prefill's last wave leaves idle.  Either batch
  * may be NULL or empty (then this is the plain call on `stream`).  The two
  * workspaces must be distinct buffers (LAZY_EINVAL otherwise).  Calls are
  * serialised on the host by a mutex.  The fork and join are event waits, so

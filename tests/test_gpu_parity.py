@@ -469,8 +469,9 @@ def test_mixed_step_equals_separate_calls_and_the_oracle(hq, hkv):
 
 
 def test_mixed_step_orders_work_on_the_callers_stream():
-    """Work enqueued on the caller's stream after the call sees both outputs (the join), and the
-    side stream does not start before work enqueued before the call (the fork)."""
+    """Work enqueued on the caller's stream after the call sees both outputs (the join), and
+    neither batch starts before work enqueued before the call (the fork of the library's side
+    stream, which runs the prefill, and stream order for the decode)."""
     case = _mixed_case()
     dc_ = DeviceCase(case)
     pf, dc = dc_.mixed_batches(3)
@@ -479,7 +480,8 @@ def test_mixed_step_orders_work_on_the_callers_stream():
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
         torch.cuda._sleep(2_000_000)         # the caller's stream is still busy at the fork ...
-        dc["out"].fill_(7.0)                 # ... with a write the decode must come after
+        dc["out"].fill_(7.0)                 # ... with writes the decode and the prefill must
+        pf["out"].fill_(7.0)                 # come after
         dc_.mixed(pf, dc, stream=s)
         got_dc = dc["out"].clone()           # after the call, on the caller's stream
         got_pf = pf["out"].clone()
