@@ -66,11 +66,11 @@ TRAFFIC = {
     # ncu --clock-control none --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
     #     -k regex:decode_split -s 3 -c 1
     #     python bench.py --steps 2 --warmup 3 --no-cpu --no-compare --no-e2e --no-distinct
-    "decode_8b": {"sha": "545dbebd3d15d2f3", "bytes": 786657024 + 6874112},
+    "decode_8b": {"sha": "b4ca7d6410749acd", "bytes": 786105600 + 7165184},
     # the same command with --no-prefill --workload decode_8b_distinct
-    "decode_8b_distinct": {"sha": "545dbebd3d15d2f3", "bytes": 1095635456 + 7873024},
+    "decode_8b_distinct": {"sha": "b4ca7d6410749acd", "bytes": 1095527424 + 6870272},
     # the first command with -k regex:prefill_tc
-    "prefill_8b": {"sha": "196b11b5ee72ba24", "bytes": 301056000 + 26041344},
+    "prefill_8b": {"sha": "1711e2f3f2c20df9", "bytes": 300517888 + 26762752},
 }
 
 
