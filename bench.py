@@ -621,7 +621,7 @@ def run_extended(args, world, peaks, peak_src, flush):
             kept[step.kind] = ds
         if "prefill" in kept and "decode" in kept:
             # the whole serving step: the two attention calls back to back on one stream, and the
-            # same two batches in one lazy_mixed_attn call (decode on the side stream)
+            # same two batches in one lazy_mixed_attn call
             pf, dc = kept["prefill"], kept["decode"]
 
             def seq(ev):

@@ -99,11 +99,9 @@ cudaError_t launch_decode_combine(const AttnParams &p, cudaStream_t s);
 // tk, tv: the K source and V pool as rows of 128 bf16 (one box = half of one block);
 // tk8, tv8: the same memory as (d, token, head, block) (one box = half of 8 consecutive blocks);
 // tq: p.q_prep as rows of 128 bf16 (one box = half of 128 rows), used when p.q_prep is set.
-// started (optional): recorded on s just before the attention kernel (after the query
-// preparation kernel).
 cudaError_t launch_prefill_tc(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8,
                               const CUtensorMap &tv8, const CUtensorMap &tq, const AttnParams &p, bool plain,
-                              cudaStream_t s, cudaEvent_t started = nullptr);
+                              cudaStream_t s);
 constexpr int kPrefillRows = 256;   // query rows per prefill CTA
 // Units of the last, partial wave that are split in two when that wave is at most half full
 // (one prefill CTA per SM): the grid then ends with two half-length CTAs per such unit.

@@ -884,7 +884,7 @@ __global__ void __launch_bounds__(256) prefill_qprep_kernel(const AttnParams p, 
 
 template <int MODE>
 cudaError_t launch_t(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8, const CUtensorMap &tv8,
-                     const CUtensorMap &tq, const AttnParams &p, cudaStream_t s, cudaEvent_t started) {
+                     const CUtensorMap &tq, const AttnParams &p, cudaStream_t s) {
     auto kern = prefill_tc_kernel<MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
     if (e != cudaSuccess) return e;
@@ -892,10 +892,6 @@ cudaError_t launch_t(const CUtensorMap &tk, const CUtensorMap &tv, const CUtenso
     if (p.q_prep) {
         prefill_qprep_kernel<<<dim3(p.pf_mtiles * (kRows / 32), p.num_req), 256, 0, s>>>(p, MODE == kPlain);
         e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    if (started) {
-        e = cudaEventRecord(started, s);
         if (e != cudaSuccess) return e;
     }
     kern<<<p.pf_base + 2 * p.pf_nsplit, kThreads, kTcSmem, s>>>(tk, tv, tk8, tv8, tq, p);
@@ -909,10 +905,9 @@ cudaError_t launch_t(const CUtensorMap &tk, const CUtensorMap &tv, const CUtenso
 
 cudaError_t launch_prefill_tc(const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &tk8,
                               const CUtensorMap &tv8, const CUtensorMap &tq, const AttnParams &p, bool plain,
-                              cudaStream_t s, cudaEvent_t started) {
-    if (plain) return launch_t<kPlain>(tk, tv, tk8, tv8, tq, p, s, started);
-    return p.alibi ? launch_t<kAlibi>(tk, tv, tk8, tv8, tq, p, s, started)
-                   : launch_t<kLazy>(tk, tv, tk8, tv8, tq, p, s, started);
+                              cudaStream_t s) {
+    if (plain) return launch_t<kPlain>(tk, tv, tk8, tv8, tq, p, s);
+    return p.alibi ? launch_t<kAlibi>(tk, tv, tk8, tv8, tq, p, s) : launch_t<kLazy>(tk, tv, tk8, tv8, tq, p, s);
 }
 
 }  // namespace lazy

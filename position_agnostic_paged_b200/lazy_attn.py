@@ -245,8 +245,8 @@ def _nbytes(t) -> int:
 def mixed_attn(cfg: Cfg, prefill: dict | None, decode: dict | None, blk_meta, k_pool, v_pool, d_status=None,
                stream=None):
     """One serving step with prefill chunks and decodes (lazy_mixed_attn): the results of
-    prefill_attn(**prefill) and decode_attn(**decode); the decode runs on the library's side stream,
-    forked from and joined back into `stream`.
+    prefill_attn(**prefill) and decode_attn(**decode), both batches validated before either runs,
+    then run in that order on `stream`.
 
     prefill: dict(q_raw, cu_q, q_pos0, max_q, table, table_indptr, max_words, out, workspace);
     decode: dict(q_raw, q_pos, table, table_indptr, max_words, out, workspace).  The two

@@ -469,9 +469,8 @@ def test_mixed_step_equals_separate_calls_and_the_oracle(hq, hkv):
 
 
 def test_mixed_step_orders_work_on_the_callers_stream():
-    """Work enqueued on the caller's stream after the call sees both outputs (the join), and
-    neither batch starts before work enqueued before the call (the fork of the library's side
-    stream, which runs the prefill, and stream order for the decode)."""
+    """Work enqueued on the caller's stream after the call sees both outputs, and neither batch
+    starts before work enqueued before the call."""
     case = _mixed_case()
     dc_ = DeviceCase(case)
     pf, dc = dc_.mixed_batches(3)
@@ -479,7 +478,7 @@ def test_mixed_step_orders_work_on_the_callers_stream():
     dc_.separate(ref_pf, ref_dc)
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
-        torch.cuda._sleep(2_000_000)         # the caller's stream is still busy at the fork ...
+        torch.cuda._sleep(2_000_000)         # the caller's stream is still busy at the call ...
         dc["out"].fill_(7.0)                 # ... with writes the decode and the prefill must
         pf["out"].fill_(7.0)                 # come after
         dc_.mixed(pf, dc, stream=s)
