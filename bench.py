@@ -35,8 +35,8 @@ the time is the maximum over ranks and the work the sum over ranks.
 mixed 8B serving step (GQA and MQA), with the whole step timed as two calls
 and as one lazy_mixed_attn call.  --cache-sim runs the host-side cache-hit
 simulation of position-agnostic, position-aware and prefix caching (no GPU).
---profile-case launches only the attention kernel of a small case, for
-profiler captures.
+--profile-case launches only the attention kernel of a small case (or of
+the mixed 8B MQA step's decode batch), for profiler captures.
 """
 from __future__ import annotations
 
@@ -712,9 +712,10 @@ def run_reference(args):
 
 
 def run_profile_case(args):
-    """A small case for profiler captures: 2 prefill requests (64 CTAs) or 8 decode requests of the
-    8B shapes over a 100-document pool, or 32 decode requests of the MQA shapes (Hq 32, Hkv 1) over
-    a 400-document pool; the attention kernel launched --steps times."""
+    """A case for profiler captures: 2 prefill requests (64 CTAs) or 8 decode requests of the 8B
+    shapes over a 100-document pool, or 32 decode requests of the MQA shapes (Hq 32, Hkv 1) over a
+    400-document pool; or the whole decode batch of the mixed 8B MQA step (192 requests, 1 GiB
+    pool), for one-pass counters only; the attention kernel launched --steps times."""
     import torch
     from position_agnostic_paged_b200 import workloads as W
     from position_agnostic_paged_b200.runner import DevicePool, DeviceStep
@@ -722,8 +723,10 @@ def run_profile_case(args):
         wl = W.make("prefill_8b", n_docs=100, n_prefill=2)
     elif args.profile_case == "decode_small":
         wl = W.make("decode_8b", n_docs=100, n_decode=8)
-    else:
+    elif args.profile_case == "decode_mqa_small":
         wl = W.make("mixed_8b_mqa", n_docs=400, n_prefill=0, n_decode=32)
+    else:
+        wl = W.make("mixed_8b_mqa")   # its decode step only
     pool = DevicePool(wl).setup()
     ds = DeviceStep(pool, [st for st in wl.steps if st.kind == ("prefill" if "prefill" in args.profile_case
                                                                     else "decode")][0])
@@ -770,7 +773,7 @@ def main():
                     help="skip the decode step over documents shared by no two requests")
     ap.add_argument("--extended", action="store_true",
                     help="also time decode 70B (Zipf 1.2 and uniform) and the mixed 8B step (GQA, MQA)")
-    ap.add_argument("--profile-case", choices=["prefill_small", "decode_small", "decode_mqa_small"],
+    ap.add_argument("--profile-case", choices=["prefill_small", "decode_small", "decode_mqa_small", "decode_mqa_full"],
                     help="launch only the attention kernel of a small case --steps times (for ncu captures; "
                          "prints no result line)")
     ap.add_argument("--cache-sim", action="store_true",
