@@ -130,6 +130,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
     const uint32_t *tbl = p.table + wbase;
     const int qpos = p.q_pos[r];
 
+    // The K producer's first table words, loaded before the barrier set-up.
+    uint32_t first_wl = 0xFFFFFFFFu;
+    if (warp == 0 && lane < kTB && lo + lane < hi) first_wl = tbl[lo + lane];
+
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&bars[B_KFULL + i], 1);
@@ -172,7 +176,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
         int issued = 0;
         for (int w = lo, j = 0; w < hi; ++j) {
             // the tile: up to 8 consecutive words sharing one offset; lane k < 8 holds word k
-            const uint32_t wl = (lane < kTB && w + lane < hi) ? tbl[w + lane] : 0xFFFFFFFFu;
+            const uint32_t wl = j == 0 ? first_wl : ((lane < kTB && w + lane < hi) ? tbl[w + lane] : 0xFFFFFFFFu);
             const int off = word_offset(__shfl_sync(0xffffffffu, wl, 0));
             const bool same = lane < kTB && w + lane < hi && word_offset(wl) == off;
             const int n = __ffs(~__ballot_sync(0xffffffffu, same)) - 1;   // lanes 0..n-1 share it
@@ -369,25 +373,51 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
         // Q'_h = R(q_pos - o) q_h * scale_log2 for each new offset o (once, by q_pos, on the plain
         // path; the identity under ALiBi), lane h writing head h's row of the MMA A operand
         // (K-major, 128-byte swizzle, two 64-column half planes).  The angles are evaluated once
-        // per rotation, two per lane, and shared through shared memory.
+        // per rotation, two per lane, and shared through shared memory.  The raw query row is
+        // loaded once and kept in registers, and the first query is made from the first table
+        // word, read here, before the tile information is published (the issuer sees the same
+        // offset in the first entry): it is ready about when the first K tile lands.
+        uint4 qa[8], qb[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            qa[c] = make_uint4(0, 0, 0, 0);
+            qb[c] = make_uint4(0, 0, 0, 0);
+        }
+        int first_rot = PLAIN ? 0 : qpos;
+        if (lo < hi) {
+            if (lane < G) {
+                const uint4 *qrow = reinterpret_cast<const uint4 *>(
+                    p.q_raw + (static_cast<size_t>(r) * p.hq + kvh * G + lane) * kHeadDim);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    qa[c] = __ldg(qrow + c);       // elements 8c .. 8c + 7
+                    qb[c] = __ldg(qrow + 8 + c);   // elements 64 + 8c ..
+                }
+            }
+            if (!PLAIN && !ALIBI) first_rot = word_offset(tbl[lo]);
+        }
         int gen = -1, cur_rot = INT_MIN;
-        const uint4 *qrow =
-            reinterpret_cast<const uint4 *>(p.q_raw + (static_cast<size_t>(r) * p.hq + kvh * G + lane) * kHeadDim);
         const float sc = p.scale_log2;
-        for (int w = lo, j = 0; w < hi; ++j) {
-            const int is = j % kInfo;
-            if (!wwait(&bars[B_IFULL + is], (j / kInfo) & 1, abort_flag, p.d_status)) break;
-            const int n = info[is].n, off = info[is].off;
-            __syncwarp();
-            if (leader) mbar_arrive(&bars[B_IEMPTY + is]);
-            w += n;
-            const int rot = PLAIN ? 0 : (ALIBI ? qpos : off);
+        bool first = true;
+        for (int w = lo, j = 0; w < hi;) {
+            int rot = first_rot;
+            if (!first) {
+                const int is = j % kInfo;
+                if (!wwait(&bars[B_IFULL + is], (j / kInfo) & 1, abort_flag, p.d_status)) break;
+                const int n = info[is].n, off = info[is].off;
+                __syncwarp();
+                if (leader) mbar_arrive(&bars[B_IEMPTY + is]);
+                w += n;
+                ++j;
+                rot = PLAIN ? 0 : (ALIBI ? qpos : off);
+            }
+            first = false;
             if (rot == cur_rot) continue;
             cur_rot = rot;
             ++gen;
-            // The new query is computed into registers as soon as its tile's information appears
-            // (up to the ring's depth ahead of the MMAs); only the store waits until the previous
-            // query is no longer read (every MMA issued before QFREE completed).
+            // The new query is computed into registers as soon as its offset is known; only the
+            // store waits until the previous query is no longer read (every MMA issued before
+            // QFREE completed).
             const int delta = qpos - rot;
             float c0, s0, c1, s1;
             rope_cos_sin(delta, p.rope.theta[lane], c0, s0);
@@ -403,16 +433,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
                 hi8[c] = make_uint4(0, 0, 0, 0);
             }
             if (lane < G) {
-                uint4 a8[8], b8[8];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    a8[c] = __ldg(qrow + c);       // elements 8c .. 8c + 7
-                    b8[c] = __ldg(qrow + 8 + c);   // elements 64 + 8c ..
+                    // keeps the unpacked, scaled query from being hoisted out of the loop (128
+                    // floats held across it would not fit the registers)
+                    asm volatile("" : "+r"(qa[c].x), "+r"(qa[c].y), "+r"(qa[c].z), "+r"(qa[c].w));
+                    asm volatile("" : "+r"(qb[c].x), "+r"(qb[c].y), "+r"(qb[c].z), "+r"(qb[c].w));
                 }
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const uint32_t *aw = reinterpret_cast<const uint32_t *>(&a8[c]);
-                    const uint32_t *bw = reinterpret_cast<const uint32_t *>(&b8[c]);
+                    const uint32_t *aw = reinterpret_cast<const uint32_t *>(&qa[c]);
+                    const uint32_t *bw = reinterpret_cast<const uint32_t *>(&qb[c]);
                     uint32_t *lw = reinterpret_cast<uint32_t *>(&lo8[c]);
                     uint32_t *hw = reinterpret_cast<uint32_t *>(&hi8[c]);
 #pragma unroll
