@@ -77,7 +77,8 @@ constexpr int B_KFULL = 0, B_KEMPTY = B_KFULL + kStages, B_VFULL = B_KEMPTY + kS
               kBars = B_DRAIN + 1;
 constexpr int kOffCs = kOffBar + kBars * 8;         // cos, sin of the 64 rotation angles (float2)
 constexpr int kOffMisc = kOffCs + kHalfDim * 8;     // tensor-memory address, abort flag
-constexpr int kSmemUse = kOffMisc + 16;
+constexpr int kOffTheta = kOffMisc + 16;            // the 64 rotation frequencies (double)
+constexpr int kSmemUse = kOffTheta + kHalfDim * 8;
 constexpr size_t kSmemTc = kSmemUse + 1024;
 static_assert(kSmemTc <= 232448, "shared memory budget");
 // consumers of a tile-information entry: the V producer, the issuer, the rotation warp, both
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
     float2 *cs = reinterpret_cast<float2 *>(sm + kOffCs);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);
+    double *theta_s = reinterpret_cast<double *>(sm + kOffTheta);
 
     const int split = blockIdx.x, kvh = blockIdx.y, r = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -130,9 +132,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
     const uint32_t *tbl = p.table + wbase;
     const int qpos = p.q_pos[r];
 
-    // The K producer's first table words, loaded before the barrier set-up.
+    // The K producer's first table words, loaded before the barrier set-up; the two idle warps
+    // copy the rotation frequencies to shared memory meanwhile (per-lane reads of the parameter
+    // table serialise, so the rotation warp does not make them).
     uint32_t first_wl = 0xFFFFFFFFu;
     if (warp == 0 && lane < kTB && lo + lane < hi) first_wl = tbl[lo + lane];
+    if (warp >= 6) theta_s[32 * (warp - 6) + lane] = p.rope.theta[32 * (warp - 6) + lane];
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -373,7 +378,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
         // Q'_h = R(q_pos - o) q_h * scale_log2 for each new offset o (once, by q_pos, on the plain
         // path; the identity under ALiBi), lane h writing head h's row of the MMA A operand
         // (K-major, 128-byte swizzle, two 64-column half planes).  The angles are evaluated once
-        // per rotation, two per lane, and shared through shared memory.  The raw query row is
+        // per rotation, two per lane (frequencies from shared memory), and shared through shared
+        // memory.  The raw query row is
         // loaded once and kept in registers, and the first query is made from the first table
         // word, read here, before the tile information is published (the issuer sees the same
         // offset in the first entry): it is ready about when the first K tile lands.
@@ -420,8 +426,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(const __grid_c
             // QFREE completed).
             const int delta = qpos - rot;
             float c0, s0, c1, s1;
-            rope_cos_sin(delta, p.rope.theta[lane], c0, s0);
-            rope_cos_sin(delta, p.rope.theta[lane + 32], c1, s1);
+            rope_cos_sin(delta, theta_s[lane], c0, s0);
+            rope_cos_sin(delta, theta_s[lane + 32], c1, s1);
             __syncwarp();   // the previous rotation's reads of the angle table are done
             cs[lane] = make_float2(c0, s0);
             cs[lane + 32] = make_float2(c1, s1);
