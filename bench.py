@@ -70,7 +70,7 @@ TRAFFIC = {
     # the same command with --no-prefill --workload decode_8b_distinct
     "decode_8b_distinct": {"sha": "b4ca7d6410749acd", "bytes": 1095527424 + 6870272},
     # the first command with -k regex:prefill_tc
-    "prefill_8b": {"sha": "1711e2f3f2c20df9", "bytes": 300517888 + 26762752},
+    "prefill_8b": {"sha": "048840e346fb33b7", "bytes": 302145280 + 26523392},
 }
 
 
