@@ -36,6 +36,7 @@
 //   warp 5   softmax of stream 1: lanes 32-63 (rows 32-63, the second copy of
 //            the heads), so that the two streams' softmaxes run on different
 //            sub-partitions of the SM
+//   warps 6-7 copy the 64 rotation frequencies to shared memory at the start
 // Tensor memory (512 columns): S0 [0,128) (P0 = its first 64 columns),
 // S1 [128,256) (P1), O0 [256,384), O1 [384,512).
 #include <climits>
