@@ -398,10 +398,9 @@ DecodePlan decode_plan(int num_req, int hkv, int max_words, int group) {
     const int units = max(1, num_req * hkv);
     const bool tc = group >= kDecodeTcMinGroup;
     // warp-MMA kernels: about 2000 CTAs (several waves over 148 SMs at ~3 resident CTAs each),
-    // at least 8 words (128 keys) per split; tensor-memory kernel (one CTA per SM): about 444
-    // CTAs (three waves over 148 SMs: each CTA's fill and drain costs about as much as five
-    // key tiles, so fewer, longer CTAs pay), at least 16 words (two key tiles) per split
-    const int target = tc ? 444 : 2048;
+    // at least 8 words (128 keys) per split; tensor-memory kernel (one CTA per SM): about 600
+    // CTAs, at least 16 words (two key tiles) per split
+    const int target = tc ? 592 : 2048;
     const int min_words = tc ? 16 : 8;
     int splits = (target + units - 1) / units;
     const int max_splits = max(1, (max_words + min_words - 1) / min_words);

@@ -45,8 +45,8 @@ def test_the_benchmark_decode_shapes_fit_the_array():
     of 512 tokens and a 64-token question plus the new token), decode 70B and its uniform variant
     (128 requests, 32 x 512 + 128 + 1), and the mixed 8B step's decodes (192 requests, 8 documents
     of at most 2048 tokens + 64 + 1).  The MQA variant of the mixed step does not fit: its 192
-    requests with one KV head run on the tensor-memory decode kernel as 3 CTAs of two softmax
-    streams each, 6 partials of 32 query heads per request (about 19 MB), and the entry point
+    requests with one KV head run on the tensor-memory decode kernel as 4 CTAs of two softmax
+    streams each, 8 partials of 32 query heads per request (about 26 MB), and the entry point
     refuses it before launching anything."""
     cap = la.decode_noalloc_capacity()
     shapes = [(la.Cfg(32, 8), 64, _words([512] * 8, 65)),
